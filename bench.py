@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of zero-copy host/HBM split-KV decode attention on B200.
+
+One step = one dkv_attn_decode call over one batch of the workload: the
+zero-copy host-stream kernel (aux stream), the HBM split-K kernel and the LSE
+merge.  Default workload: the LLaMA-3-8B-shaped layer (B=8, Hq=32, Hkv=8,
+D=128, L=32768, bf16 K/V, 16-token blocks, half the blocks of each sequence
+in mapped pinned host memory, chosen at random).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dkv|reference]
+
+With N > 1 (launched by torchrun) every rank runs an independent replica of
+the workload on its own GPU and PCIe link; rank 0 prints the JSON line with
+the device time taken as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kvgen  # noqa: E402
+
+METRIC = "decode-attention µs/step & KV GB/s, fraction of PCIe+HBM roofline"
+HBM_NOMINAL_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama3_8b")
+    ap.add_argument("--impl", choices=("dkv", "reference"), default="dkv")
+    ap.add_argument("--host-ctas", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def workload_for_rank(name: str, rank: int) -> kvgen.Workload:
+    """Replica r draws its own inputs: same shapes and recipe, seed + 1000 r."""
+    w = kvgen.get(name)
+    return w if rank == 0 else w.replace(seed=w.seed + 1000 * rank)
+
+
+# ----------------------------------------------------------------------------- measurements
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while active."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(", ") for r in self.file.read().splitlines() if r.strip()]
+        self.file.close()
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.strip() == "Active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def measure_pcie_gbs(device, nbytes: int = 1 << 30, reps: int = 5) -> float:
+    """Pinned host -> device cudaMemcpyAsync bandwidth (the PCIe roofline denominator)."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    s = torch.cuda.current_stream(device)
+    best = float("inf")
+    for i in range(reps + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        dst.copy_(src, non_blocking=True)
+        b.record(s)
+        b.synchronize()
+        if i:
+            best = min(best, a.elapsed_time(b))
+    del src, dst
+    return nbytes / (best * 1e-3) / 1e9
+
+
+def measured_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
+
+
+def kernel_source_sha() -> str:
+    with open(os.path.join(ROOT, "decode_attention_host_b200", "csrc", "dkv_kernels.cuh"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """ncu DRAM + sysmem bytes per launch from profiles/traffic.json, if taken on the current kernel source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(f"{kernel}:{workload}")
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return rec
+
+
+def oracle_gbs(w: kvgen.Workload, q, k, v, lens, group_mask) -> tuple[float, float, int]:
+    """Time the fp64 oracle on the (batch, kv head) groups of group_mask: (GB/s, seconds, threads)."""
+    import oracle
+    dt = oracle.KV_BF16 if w.kv_dtype == kvgen.BF16 else oracle.KV_F16
+    t0 = time.perf_counter()
+    oracle.decode(q, k, v, lens, dt, w.rope_base, group_mask=group_mask)
+    sec = time.perf_counter() - t0
+    tokens = sum(int(lens[b]) for b in range(w.batch) for h in range(w.num_kv_heads) if group_mask[b, h])
+    nbytes = tokens * 2 * w.head_dim * 2
+    return nbytes / sec / 1e9, sec, oracle.num_threads()
+
+
+# ----------------------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    w = kvgen.get(args.workload)
+    lens = kvgen.gen_seq_lens(w)
+    q = kvgen.gen_q(w)
+    k, v = kvgen.gen_kv(w, lens)
+    threads = oracle.num_threads()
+    ngroups = w.batch * w.num_kv_heads
+    per_step = max(1, min(ngroups, threads))
+    order = np.random.default_rng(0).permutation(ngroups)
+    times, nbytes = [], []
+    for i in range(args.warmup + args.steps):
+        mask = np.zeros((w.batch, w.num_kv_heads), dtype=np.uint8)
+        for g in order[(i * per_step) % ngroups:][:per_step]:
+            mask.flat[g] = 1
+        gbs, sec, _ = oracle_gbs(w, q, k, v, lens, mask)
+        if i >= args.warmup:
+            times.append(sec)
+            nbytes.append(gbs * sec * 1e9)
+    value = sum(nbytes) / sum(times) / 1e9
+    total_bytes = float(lens.astype(np.int64).sum()) * w.num_kv_heads * 2 * w.head_dim * 2
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_bytes / (value * 1e9), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{per_step} of {ngroups} (batch, kv head) groups per step; ms_per_step "
+                                   f"extrapolates to the whole batch"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: kvgen.Workload, n: int) -> dict:
+    return {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "seq_len": w.ctx if not isinstance(w.ctx, tuple) else list(w.ctx),
+            "block_size": w.block_size, "kv_dtype": w.kv_dtype, "rope_base": w.rope_base,
+            "placement": w.placement, "host_fraction": w.host_fraction,
+            "parallelism": "replicas" if n > 1 else "single_gpu"}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_dkv(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init("nccl")
+    import decode_attention_host_b200 as dkv
+
+    w = workload_for_rank(args.workload, rank)
+    q = kvgen.gen_q(w)
+    lens = kvgen.gen_seq_lens(w)
+    k, v = kvgen.gen_kv(w, lens)
+    placement = dkv.DKV_PLACE_PREFIX_HOST if w.placement == "prefix_host" else dkv.DKV_PLACE_RANDOM
+    kv = dkv.PagedKV(k, v, lens, w.block_size, placement, w.host_fraction, w.shuffle, w.seed, device=local)
+    attn = dkv.DecodeAttention(w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                               dkv.DKV_KV_BF16 if w.kv_dtype == kvgen.BF16 else dkv.DKV_KV_F16, w.rope_base,
+                               w.batch, kv.stride, device=local, host_ctas=args.host_ctas)
+    keep_logical = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if not keep_logical:
+        del k, v
+    q_dev = torch.from_numpy(q).to(device)
+    out = torch.empty_like(q_dev)
+    stream = torch.cuda.current_stream(device)
+    b_pcie = measure_pcie_gbs(device)
+
+    for _ in range(args.warmup):
+        attn(q_dev, kv, out, stream)
+    torch.cuda.synchronize(device)
+    if attn.status() != 0:
+        raise RuntimeError("device status nonzero after warm-up")
+
+    # ---- timed region: K steps, device time on the launching stream, per-kernel events inside the library
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier()
+    torch.cuda.synchronize(device)
+    clocks.start()
+    dkv.dkv_profile_begin(attn.handle, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        attn(q_dev, kv, out, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    kernel_ms, kernel_counts = dkv.dkv_profile_end(attn.handle)
+    clock_info = clocks.stop()
+    barrier()
+    launches_per_step = attn.launches()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local, device)
+
+    # ---- end to end through the public API: inputs from pinned host memory, result back to the host
+    e2e = None
+    if not args.no_e2e:
+        q_h = torch.from_numpy(q).pin_memory()
+        lens_h = torch.from_numpy(kv.seq_lens).pin_memory()
+        table_h = torch.from_numpy(kv.table).pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = q_h.numel() * 4 + lens_h.numel() * 4 + table_h.numel() * 4
+        d2h = out_h.numel() * 4
+
+        def e2e_step():
+            q_dev.copy_(q_h, non_blocking=True)
+            kv.seq_lens_dev.copy_(lens_h, non_blocking=True)
+            kv.table_dev.copy_(table_h, non_blocking=True)
+            attn(q_dev, kv, out, stream)
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, device)
+        e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms}
+
+    if rank != 0:
+        barrier()
+        kv.free()
+        return 0
+
+    # ---- sampled parity: the fp64 oracle on two (batch, kv head) groups
+    parity = None
+    if keep_logical:
+        import oracle
+        mask = np.zeros((w.batch, w.num_kv_heads), dtype=np.uint8)
+        mask[0, 0] = mask[-1, -1] = 1
+        want = oracle.decode(q, k, v, lens, oracle.KV_BF16 if w.kv_dtype == kvgen.BF16 else oracle.KV_F16,
+                             w.rope_base, group_mask=mask)
+        got = out.cpu().numpy()
+        rows = np.repeat(mask.astype(bool), w.group_size, axis=1)
+        parity = {"groups": int(mask.sum()), "max_abs_err": float(np.abs(got[rows] - want[rows]).max()),
+                  "tolerance": 2e-3}
+
+    host_bytes, dev_bytes = kv.host_bytes, kv.dev_bytes
+    total = (host_bytes + dev_bytes) * world
+    value = total / (ms * 1e-3) / 1e9
+    peaks = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    hbm_src = "MEASURED_PEAKS.json hbm_gbs (copy, measured)" if "hbm_gbs" in peaks else "fallback 6650 GB/s"
+
+    kernels = []
+    for idx, name, nbytes, bound, peak, unit_src in (
+            (0, "host_stream", host_bytes, "pcie", b_pcie, "pinned H2D cudaMemcpyAsync measured in this run"),
+            (1, "hbm_split_k", dev_bytes, "hbm", hbm_peak, hbm_src)):
+        if kernel_counts[idx] == 0:
+            continue
+        avg_ms = kernel_ms[idx] / kernel_counts[idx]
+        achieved = nbytes / (avg_ms * 1e-3) / 1e9
+        traffic = recorded_traffic(name, w.name)
+        kernels.append({"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "peak_source": unit_src, "avg_ms": avg_ms,
+                        "algorithmic_bytes_per_launch": nbytes,
+                        "traffic": traffic.get("bytes_per_launch") if traffic else None,
+                        "traffic_detail": traffic})
+    dominant = max(kernels, key=lambda r: r["avg_ms"]) if kernels else None
+    t_star_meas = max(host_bytes / (b_pcie * 1e9), dev_bytes / (hbm_peak * 1e9))
+    t_star_nom = max(host_bytes / (b_pcie * 1e9), dev_bytes / (HBM_NOMINAL_GBS * 1e9))
+
+    cpu = None
+    if keep_logical:
+        ngroups = w.batch * w.num_kv_heads
+        mask = np.ones((w.batch, w.num_kv_heads), dtype=np.uint8)
+        gbs, sec, threads = oracle_gbs(w, q, k, v, lens, mask)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"all {ngroups} (batch, kv head) groups of one step, {sec:.1f} s"}
+
+    if e2e is not None:
+        e2e["value"] = total / (e2e["ms_per_step"] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+        "config": dict(workload_config(w, world), host_bytes=host_bytes, dev_bytes=dev_bytes,
+                       l2="inputs larger than L2: %.0f MiB of KV per step vs 126 MB L2" % ((host_bytes + dev_bytes) / 2**20)),
+        "roofline": ({k2: dominant[k2] for k2 in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+                     if dominant else None),
+        "roofline_kernels": kernels,
+        "roofline_step": {"t_star_ms_measured_hbm": t_star_meas * 1e3, "frac_measured_hbm": t_star_meas / (ms * 1e-3),
+                          "t_star_ms_nominal_hbm": t_star_nom * 1e3, "frac_nominal_hbm": t_star_nom / (ms * 1e-3),
+                          "b_pcie_gbs": b_pcie, "b_hbm_measured_gbs": hbm_peak, "b_hbm_nominal_gbs": HBM_NOMINAL_GBS},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clock_info,
+        "cpu_baseline": cpu,
+        "parity": parity,
+    }
+    print(json.dumps(line), flush=True)
+    barrier()
+    kv.free()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    rc = run_dkv(args)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

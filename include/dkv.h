@@ -1,0 +1,222 @@
+/*
+ * dkv.h -- C ABI of libdkv: single-token decode attention (GQA/MHA, NeoX
+ * RoPE) over a paged KV cache split between CPU-pinned host memory and GPU
+ * HBM, for NVIDIA B200 (sm_100a).
+ *
+ * Method (DirectKV README, opening summary and Attribution; SplitKernel
+ * README, Overview and Key Features): the KV cache of a sequence is split at
+ * block granularity between host memory and device memory.  Host-resident
+ * blocks are read by the GPU directly from mapped pinned memory into shared
+ * memory, with no staging copy in HBM; device-resident blocks are read from
+ * HBM.  Each side produces split-K partial results (an un-normalised
+ * attention output and a log-sum-exp per query head and split), and a merge
+ * combines all partials into the exact softmax attention output.
+ *
+ * Conventions shared by every entry point:
+ *   - Every function returns DKV_OK (0) or a negative DKV_ERR_* code; the
+ *     message of the last failure on the calling thread is available from
+ *     dkv_last_error_string().  No function aborts or throws.
+ *   - "device pointer": memory the GPU of the handle can read or write
+ *     (cudaMalloc'd, or the device alias of mapped pinned host memory).
+ *     "host pointer": ordinary CPU memory.
+ *   - K/V element storage is 16-bit (IEEE binary16 or bfloat16), stored
+ *     UN-ROTATED; the library applies RoPE to keys as it reads them.
+ *   - Paged pool layout, for both pools: [num_blocks][Hkv][block_size][D],
+ *     row-major; one (block, kv head) tile is block_size*D contiguous elements.
+ *   - Logical positions: token t of a sequence is at position t; the query of
+ *     a sequence of length L is at position L.
+ *   - Query head hq reads KV head hq / G, G = Hq / Hkv (consecutive groups).
+ */
+#ifndef DKV_H
+#define DKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DKV_API __attribute__((visibility("default")))
+#else
+#define DKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ------------------------------------------------------ */
+#define DKV_OK 0
+#define DKV_ERR_INVALID_ARG (-1) /* a pointer, size or enum is out of its documented range */
+#define DKV_ERR_UNSUPPORTED (-2) /* valid request this build does not implement (head dim, group size) */
+#define DKV_ERR_CUDA (-3)        /* a CUDA runtime call failed; see dkv_last_error_string() */
+#define DKV_ERR_NO_MEMORY (-4)   /* device or pinned host allocation failed */
+
+/* ---- device-side status bits (read with dkv_get_status) ----------------- */
+#define DKV_STATUS_BAD_BLOCK_ID 1 /* a block table entry is outside both pools */
+#define DKV_STATUS_BAD_SEQ_LEN 2  /* seq_lens[b] < 0 or beyond the table / handle capacity */
+
+typedef enum { DKV_KV_F16 = 0, DKV_KV_BF16 = 1 } dkv_kv_dtype;
+
+typedef struct dkv_config {
+  int32_t num_q_heads;        /* Hq >= 1 */
+  int32_t num_kv_heads;       /* Hkv >= 1, Hq % Hkv == 0; G = Hq/Hkv in {1, 2, 4} */
+  int32_t head_dim;           /* D in {64, 128} */
+  int32_t block_size;         /* S tokens per block: multiple of 16, 16 <= S <= 1024 */
+  int32_t kv_dtype;           /* dkv_kv_dtype */
+  double rope_base;           /* NeoX RoPE base; 0 disables rotation */
+  double scale;               /* softmax scale; 0 means 1/sqrt(D) */
+  int32_t max_batch;          /* largest batch passed to dkv_attn_decode */
+  int32_t max_blocks_per_seq; /* largest number of blocks of one sequence */
+  int32_t device;             /* CUDA device ordinal the handle is bound to */
+  int32_t host_ctas;          /* CTAs of the zero-copy host kernel; 0 = library default (16) */
+} dkv_config;
+
+typedef struct dkv_handle dkv_handle;
+typedef struct CUstream_st* dkv_stream_t; /* the same type as cudaStream_t; NULL = legacy default stream */
+
+/*
+ * dkv_create -- validate cfg and allocate the per-handle workspace on
+ * cfg->device: the split-K partial buffers, the device status word, an
+ * auxiliary high-priority stream and two events used to fork/join the host
+ * and HBM kernels.  On success *out owns all of it until dkv_destroy.
+ * Errors: INVALID_ARG (null pointers, out-of-range fields), UNSUPPORTED
+ * (head_dim or group size), NO_MEMORY, CUDA.
+ */
+DKV_API int dkv_create(const dkv_config* cfg, dkv_handle** out);
+
+/* dkv_destroy -- synchronise the handle's streams and free everything it owns.
+ * NULL is accepted and ignored. */
+DKV_API int dkv_destroy(dkv_handle* h);
+
+/*
+ * dkv_attn_decode -- one decode-attention step for a batch of sequences.
+ *
+ *   q            device, fp32 [batch][Hq][D]: the new token's query, un-rotated.
+ *   k_host,v_host  device aliases of MAPPED pinned host memory (see
+ *                dkv_host_pool_alloc), pool layout, >= host_split blocks.
+ *                May be NULL only when host_split == 0.
+ *   k_dev,v_dev  device memory (HBM), pool layout, >= num_dev_blocks blocks.
+ *                May be NULL only when num_dev_blocks == 0.
+ *   block_table  device, int32 [batch][block_table_stride]: entry j of row b
+ *                is the physical id of logical block j (tokens j*S .. j*S+S-1)
+ *                of sequence b.  Ids in [0, host_split) index the host pool;
+ *                ids in [host_split, host_split + num_dev_blocks) index the
+ *                device pool at id - host_split.  Only entries
+ *                j < ceil(seq_lens[b]/S) are read.
+ *   seq_lens     device, int32 [batch]: context length L_b (tokens already in
+ *                the cache; the new token's own K/V are not part of it).
+ *                0 <= L_b <= min(block_table_stride, max_blocks_per_seq) * S.
+ *   out          device, fp32 [batch][Hq][D]: softmax attention output.
+ *   stream       all work is ordered on this stream (forked internally onto
+ *                the handle's auxiliary stream and joined back); the call
+ *                neither allocates nor synchronises.  One call at a time per
+ *                handle: calls that overlap on different streams race on the
+ *                handle's workspace.
+ * Host-side argument errors return INVALID_ARG / UNSUPPORTED before anything
+ * is launched.  Table entries outside both pools and out-of-range lengths are
+ * detected on the device: the status word records DKV_STATUS_* bits and the
+ * affected rows of out are written as NaN (there is no device trap).
+ */
+DKV_API int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const void* v_host,
+                    const void* k_dev, const void* v_dev, const int32_t* block_table,
+                    const int32_t* seq_lens, int32_t host_split, float* out, dkv_stream_t stream,
+                    int32_t batch, int32_t block_table_stride, int32_t num_dev_blocks);
+
+/* dkv_get_status -- synchronise the handle's device, return the accumulated
+ * DKV_STATUS_* bits in *status and clear them. */
+DKV_API int dkv_get_status(dkv_handle* h, int32_t* status);
+
+/* dkv_last_error_string -- message of the last failed call on this thread
+ * ("" if none).  The string stays valid until the next failing call. */
+DKV_API const char* dkv_last_error_string(void);
+
+/* dkv_last_launch_count -- number of kernels the handle's last successful
+ * dkv_attn_decode launched (host stream, HBM split-K, merge). */
+DKV_API int dkv_last_launch_count(const dkv_handle* h, int32_t* count);
+
+/* dkv_query_plan -- the split-K decomposition dkv_attn_decode would use for
+ * (batch, block_table_stride): splits per sequence and blocks per split. */
+DKV_API int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_table_stride, int32_t* num_splits,
+                   int32_t* blocks_per_split);
+
+/* ---- per-kernel timing ---------------------------------------------------
+ * dkv_profile_begin -- record CUDA events around every kernel of the next
+ * max_calls dkv_attn_decode calls, each on the stream that kernel runs on
+ * (the host-stream kernel runs on the handle's auxiliary stream).  Events are
+ * created here, never inside dkv_attn_decode.  Not for use while a stream is
+ * being captured into a CUDA graph.  Errors: INVALID_ARG, CUDA. */
+DKV_API int dkv_profile_begin(dkv_handle* h, int32_t max_calls);
+
+/* dkv_profile_end -- synchronise the handle's device, then return in ms[k] the
+ * summed device time of kernel k over the recorded calls and in counts[k] how
+ * many launches were recorded: k = 0 zero-copy host kernel, 1 HBM split-K
+ * kernel, 2 LSE merge.  Releases the events.  Errors: INVALID_ARG, CUDA. */
+DKV_API int dkv_profile_end(dkv_handle* h, float* ms, int32_t* counts);
+
+/* ---- host KV pool ------------------------------------------------------- */
+
+/* dkv_host_pool_alloc -- page-locked host memory that is mapped into the
+ * address space of every GPU (cudaHostAlloc Mapped|Portable).  *ptr is both
+ * the host address and, with unified addressing, the device alias to pass as
+ * k_host / v_host.  Release with dkv_host_pool_free.  Errors: INVALID_ARG,
+ * NO_MEMORY. */
+DKV_API int dkv_host_pool_alloc(size_t bytes, void** ptr);
+DKV_API int dkv_host_pool_free(void* ptr);
+
+/* ---- partitioner (host side, setup only) --------------------------------
+ * Placement of logical blocks between the host pool and the device pool
+ * (SplitKernel README, Key Features: host/device KV cache partitioning and
+ * placement / offloading-ratio utilities). */
+typedef enum {
+  DKV_PLACE_PREFIX_HOST = 0, /* the oldest round(f*n_b) blocks of each sequence on the host, the newest on HBM */
+  DKV_PLACE_RANDOM = 1       /* round(f*n_b) blocks of each sequence chosen uniformly at random for the host */
+} dkv_placement;
+
+typedef struct dkv_plan_params {
+  int32_t block_size;   /* S, as in dkv_config */
+  int32_t placement;    /* dkv_placement */
+  double host_fraction; /* f in [0, 1] */
+  int32_t shuffle_ids;  /* nonzero: physical ids are a random permutation within each pool */
+  uint64_t seed;        /* seeds the splitmix64 stream used for random choices */
+} dkv_plan_params;
+
+typedef struct dkv_plan_result {
+  int32_t host_split;     /* number of host blocks; host ids are [0, host_split) */
+  int32_t num_dev_blocks; /* device ids are [host_split, host_split + num_dev_blocks) */
+  int64_t host_tokens;    /* valid tokens placed in host blocks */
+  int64_t dev_tokens;     /* valid tokens placed in device blocks */
+} dkv_plan_result;
+
+/*
+ * dkv_plan_blocks -- build a block table for sequences of the given lengths.
+ *   seq_lens     host, int32 [batch]
+ *   block_table  host, int32 [batch][block_table_stride], written; entries
+ *                past ceil(L_b/S) are set to -1.
+ * Host blocks are numbered first (sequence-major, then logical order), then
+ * device blocks, before the optional shuffle.  Deterministic for a seed.
+ * Errors: INVALID_ARG (null pointers, f outside [0,1], a sequence that needs
+ * more than block_table_stride blocks, more than 2^31-1 blocks in total).
+ */
+DKV_API int dkv_plan_blocks(const dkv_plan_params* params, const int32_t* seq_lens, int32_t batch, int32_t* block_table,
+                    int32_t block_table_stride, dkv_plan_result* result);
+
+/*
+ * dkv_pack_kv -- write logical K/V into the paged pools following a table.
+ *   k_logical, v_logical  host, 16-bit [batch][Hkv][lmax][D]
+ *   seq_lens, block_table host, as in dkv_plan_blocks
+ *   k_host, v_host        host addresses of the host pool (>= host_split blocks)
+ *   k_dev_stage, v_dev_stage  host staging copies of the device pool
+ *                         (>= num_dev_blocks blocks) that the caller then
+ *                         copies to HBM; may be NULL when num_dev_blocks == 0.
+ * Token rows of a block past L_b are zeroed.  Errors: INVALID_ARG.
+ */
+DKV_API int dkv_pack_kv(const uint16_t* k_logical, const uint16_t* v_logical, int64_t lmax, const int32_t* seq_lens,
+                int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                const int32_t* block_table, int32_t block_table_stride, int32_t host_split,
+                int32_t num_dev_blocks, uint16_t* k_host, uint16_t* v_host, uint16_t* k_dev_stage,
+                uint16_t* v_dev_stage);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DKV_H */

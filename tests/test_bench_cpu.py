@@ -1,0 +1,65 @@
+"""bench.py host logic on the CPU: max-over-ranks timing with world size 2 (gloo),
+per-rank replica seeds, and the reference arm (the oracle) end to end."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    r, w = bench.dist_init("gloo")
+    got = bench.max_over_ranks(1.5 + 10 * rank)
+    bench.barrier()
+    seed = bench.workload_for_rank("llama3_8b", r).seed
+    q.put((r, w, got, seed))
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_with_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[2] for r in res] == [11.5, 11.5]
+    assert [r[1] for r in res] == [2, 2]
+    assert res[0][3] != res[1][3], "replicas must draw different inputs"
+
+
+def test_single_process_max_is_identity():
+    assert bench.max_over_ranks(3.25) == 3.25
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          "tiny_gqa", "--steps", "2", "--warmup", "1"], capture_output=True, text=True,
+                         timeout=300, cwd=ROOT, env=dict(os.environ, OMP_NUM_THREADS="2"))
+    assert out.returncode == 0, out.stderr
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] == 2
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["config"]["workload"] == "tiny_gqa"

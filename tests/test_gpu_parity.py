@@ -1,0 +1,208 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI (needs a B200)."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_host_b200 as dkv
+import kvgen
+from tests import gpu_cases as gc
+from tests.test_golden import load_golden
+
+pytestmark = pytest.mark.gpu
+
+
+def check(case: gc.Case, tol=gc.TOL):
+    got = case.run()
+    want = case.oracle()
+    err = gc.max_err(got, want)
+    assert case.attn.status() == 0
+    assert err <= tol, f"{case.w.name}: max abs err {err:.3e}"
+    return got, err
+
+
+def test_tiny_gqa_matches_oracle_and_golden():
+    case = gc.Case(kvgen.TINY_GQA)
+    got, err = check(case)
+    _, golden = load_golden()
+    assert np.abs(got[0] - golden).max() <= gc.TOL
+    # tokens 0..255 on the host, 256..511 in HBM: both kernels and the merge ran
+    assert case.kv.host_bytes == case.kv.dev_bytes == 256 * 2 * 64 * 2
+    assert case.attn.launches() == 3
+    case.free()
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("llama3_8b", dict(batch=2, ctx=3000)),                           # ragged tail, random half on host
+    ("long_ctx", dict(ctx=70000)),                                     # 64-token blocks, oldest 90% host
+    ("opt_6_7b", dict(batch=4, ctx=(100, 3000))),                      # MHA, ragged, shuffled ids, 75% host
+    ("opt_6_7b_norope", dict(batch=3, ctx=(20, 900), rope_base=0.0)),  # the same shape without rotation
+])
+def test_reduced_workloads(name, kw):
+    base = kvgen.get(name.replace("_norope", ""))
+    case = gc.Case(base.replace(**kw))
+    check(case)
+    case.free()
+
+
+@pytest.mark.parametrize("f", kvgen.SWEEP_HOST_FRACTION)
+def test_sweep_4k_cells_full_size(f):
+    """The 4k-context cells of the sweep at their full size (B=4, outlier keys x8)."""
+    cell = next(c for c in kvgen.sweep_cells() if c.max_ctx == 4096 and c.host_fraction == f)
+    case = gc.Case(cell)
+    check(case)
+    if f == 0.0:
+        assert case.kv.host_split == 0 and case.attn.launches() == 2
+    if f == 1.0:
+        assert case.kv.num_dev_blocks == 0 and case.attn.launches() == 2
+    case.free()
+
+
+@pytest.mark.parametrize("d,g,dt", [(64, 1, kvgen.F16), (64, 2, kvgen.BF16), (128, 1, kvgen.BF16),
+                                    (128, 2, kvgen.F16), (64, 4, kvgen.BF16), (128, 4, kvgen.F16)])
+def test_every_head_shape_and_dtype(d, g, dt):
+    w = kvgen.LLAMA3_8B.replace(name=f"shape_d{d}_g{g}", batch=3, num_kv_heads=2, num_q_heads=2 * g, head_dim=d,
+                                kv_dtype=dt, ctx=(1, 700), block_size=32, seed=40 + d + g)
+    check(gc.Case(w))
+
+
+def test_edge_lengths_in_one_batch():
+    """Empty, single-token, tile- and block-boundary and ragged sequences side by side."""
+    lens = [0, 1, 15, 16, 17, 31, 32, 33, 64, 1000]
+    w = kvgen.LLAMA3_8B.replace(name="edges", batch=len(lens), ctx=max(lens), seed=77)
+    case = gc.Case(w, lens=lens)
+    got, _ = check(case)
+    assert not got[0].any(), "an empty sequence must give a zero row"
+    case.free()
+
+
+def test_result_independent_of_placement_and_block_order():
+    w = kvgen.LLAMA3_8B.replace(name="placements", batch=2, ctx=2500, seed=91)
+    outs = []
+    for f, placement, shuffle in ((0.0, dkv.DKV_PLACE_RANDOM, False), (1.0, dkv.DKV_PLACE_RANDOM, False),
+                                  (0.37, dkv.DKV_PLACE_RANDOM, True), (0.8, dkv.DKV_PLACE_PREFIX_HOST, True),
+                                  (0.5, dkv.DKV_PLACE_RANDOM, True)):
+        case = gc.Case(w, host_fraction=f, placement=placement, shuffle=shuffle, plan_seed=int(f * 100) + 1)
+        outs.append(case.run())
+        case.free()
+    want = gc.Case(w, host_fraction=0.0).oracle()
+    for o in outs:
+        assert gc.max_err(o, want) <= gc.TOL
+        assert np.abs(o - outs[0]).max() <= 2e-5   # only fp32 summation order differs
+
+
+def test_batch_order_does_not_matter():
+    w = kvgen.OPT_6_7B.replace(name="batch_order", batch=5, ctx=(50, 600), seed=5)
+    case = gc.Case(w)
+    a = case.run()
+    perm = np.array([3, 0, 4, 1, 2])
+    w2 = w
+    case2 = gc.Case.__new__(gc.Case)
+    case2.w, case2.q, case2.lens = w2, case.q[perm].copy(), case.lens[perm].copy()
+    case2.k, case2.v = case.k[perm].copy(), case.v[perm].copy()
+    case2.kv = dkv.PagedKV(case2.k, case2.v, case2.lens, w.block_size, dkv.DKV_PLACE_RANDOM, 0.75, True, 8)
+    case2.attn = case.attn
+    case2.q_dev = torch.from_numpy(case2.q).cuda()
+    case2.out = torch.empty_like(case2.q_dev)
+    b = case2.run()
+    assert np.abs(b - a[perm]).max() <= 2e-5
+
+
+def test_repeated_calls_are_bitwise_identical_and_graph_capturable():
+    w = kvgen.LLAMA3_8B.replace(name="graph", batch=2, ctx=1500, seed=12)
+    case = gc.Case(w)
+    a = case.run()
+    b = case.run()
+    assert np.array_equal(a, b)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    case.out.fill_(float("nan"))
+    with torch.cuda.graph(g, stream=s):
+        case.attn(case.q_dev, case.kv, case.out, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(case.out.cpu().numpy(), a)
+    case.free()
+
+
+def test_bad_block_id_sets_status_and_poisons_only_its_sequence():
+    w = kvgen.LLAMA3_8B.replace(name="bad_id", batch=3, ctx=600, seed=3)
+    case = gc.Case(w)
+    good = case.run()
+    table = case.kv.table.copy()
+    table[1, 7] = case.kv.host_split + case.kv.num_dev_blocks + 5
+    case.kv.table_dev.copy_(torch.from_numpy(table))
+    out = case.run()
+    assert case.attn.status() == dkv.DKV_STATUS_BAD_BLOCK_ID
+    assert np.isnan(out[1]).all()
+    assert np.array_equal(out[[0, 2]], good[[0, 2]])
+    assert case.attn.status() == 0   # reading the status clears it
+    case.free()
+
+
+def test_bad_seq_len_sets_status():
+    w = kvgen.LLAMA3_8B.replace(name="bad_len", batch=2, ctx=300, seed=4)
+    case = gc.Case(w)
+    good = case.run()
+    lens = case.lens.copy()
+    lens[0] = case.kv.stride * w.block_size + 1
+    case.kv.seq_lens_dev.copy_(torch.from_numpy(lens))
+    out = case.run()
+    assert case.attn.status() == dkv.DKV_STATUS_BAD_SEQ_LEN
+    assert np.isnan(out[0]).all() and np.array_equal(out[1], good[1])
+    case.free()
+
+
+def test_host_side_argument_errors():
+    w = kvgen.LLAMA3_8B.replace(name="args", batch=1, ctx=200, seed=6)
+    case = gc.Case(w)
+    kv, h = case.kv, case.attn.handle
+    pageable = np.zeros(1 << 20, dtype=np.uint16)
+    args = dict(q=case.q_dev, k_host=kv.k_host.ptr, v_host=kv.v_host.ptr, k_dev=kv.k_dev, v_dev=kv.v_dev,
+                block_table=kv.table_dev, seq_lens=kv.seq_lens_dev, host_split=kv.host_split, out=case.out,
+                stream=torch.cuda.current_stream().cuda_stream, batch=1, block_table_stride=kv.stride,
+                num_dev_blocks=kv.num_dev_blocks)
+    bad = [dict(k_host=pageable), dict(k_host=kv.k_dev.data_ptr()), dict(k_dev=kv.k_host.ptr), dict(batch=2),
+           dict(block_table_stride=0), dict(host_split=-1), dict(q=None), dict(k_dev=None)]
+    for override in bad:
+        a = dict(args, **override)
+        with pytest.raises(dkv.DkvError) as e:
+            dkv.dkv_attn_decode(h, **a)
+        assert e.value.code == dkv.DKV_ERR_INVALID_ARG, override
+    dkv.dkv_attn_decode(h, **args)   # the handle still works
+    torch.cuda.synchronize()
+    case.free()
+
+
+def test_create_on_a_missing_device_fails_cleanly():
+    cfg = dkv.DkvConfig(4, 1, 64, 16, dkv.DKV_KV_F16, 1e4, 0.0, 1, 32, torch.cuda.device_count() + 3, 0)
+    hd = ctypes.c_void_p()
+    assert dkv.lib.dkv_create(ctypes.byref(cfg), ctypes.byref(hd)) == dkv.DKV_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- full sizes, bench launch config
+
+def _sampled_groups(w, n, seed):
+    rng = np.random.default_rng(seed)
+    mask = np.zeros((w.batch, w.num_kv_heads), dtype=np.uint8)
+    for i in rng.choice(w.batch * w.num_kv_heads, size=min(n, w.batch * w.num_kv_heads), replace=False):
+        mask.flat[i] = 1
+    return mask
+
+
+@pytest.mark.parametrize("name,groups", [("llama3_8b", 6), ("opt_6_7b", 6), ("long_ctx", 2)])
+def test_full_size_sampled_against_oracle(name, groups):
+    """Full-size workloads, bench launch configuration; the oracle checks sampled (batch, kv head) groups."""
+    w = kvgen.get(name)
+    case = gc.Case(w)
+    got = case.run()
+    assert np.isfinite(got).all()
+    assert case.attn.status() == 0
+    mask = _sampled_groups(w, groups, 123)
+    want = case.oracle(group_mask=mask)
+    G = w.group_size
+    rows = np.repeat(mask.astype(bool), G, axis=1)
+    err = np.abs(got[rows] - want[rows]).max()
+    assert err <= gc.TOL, f"{name}: {err:.3e}"
+    case.free()

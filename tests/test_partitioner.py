@@ -1,0 +1,126 @@
+"""The host/device block partitioner and the KV packer (host code of libdkv, no GPU)."""
+import numpy as np
+import pytest
+
+import decode_attention_host_b200 as dkv
+import kvgen
+
+
+def plan(lens, S, placement, f, shuffle=False, seed=0, stride=None):
+    lens = np.asarray(lens, dtype=np.int32)
+    stride = stride or max(1, int(-(-lens.max() // S)))
+    table = np.zeros((len(lens), stride), dtype=np.int32)
+    res = dkv.dkv_plan_blocks(dkv.DkvPlanParams(S, placement, f, int(shuffle), seed), lens, table)
+    return table, res
+
+
+def nblocks(lens, S):
+    return [int(-(-L // S)) for L in lens]
+
+
+@pytest.mark.parametrize("placement", [dkv.DKV_PLACE_PREFIX_HOST, dkv.DKV_PLACE_RANDOM])
+@pytest.mark.parametrize("shuffle", [False, True])
+def test_ids_are_a_bijection_onto_both_pools(placement, shuffle):
+    lens = [0, 1, 15, 16, 17, 1000, 333]
+    S = 16
+    table, res = plan(lens, S, placement, 0.6, shuffle, seed=11)
+    nb = nblocks(lens, S)
+    used = np.concatenate([table[b, :n] for b, n in enumerate(nb)])
+    assert sorted(used.tolist()) == list(range(sum(nb)))
+    assert res.host_split + res.num_dev_blocks == sum(nb)
+    for b, n in enumerate(nb):
+        assert (table[b, n:] == -1).all()
+        nh = int((table[b, :n] < res.host_split).sum())
+        assert nh == int(np.floor(0.6 * n + 0.5)), (b, n, nh)
+    if placement == dkv.DKV_PLACE_PREFIX_HOST:
+        for b, n in enumerate(nb):
+            host = table[b, :n] < res.host_split
+            assert not (~host[:-1] & host[1:]).any(), "a host block follows a device block"
+
+
+def test_token_counts():
+    lens = [100, 37, 64]
+    table, res = plan(lens, 32, dkv.DKV_PLACE_RANDOM, 0.5, seed=3)
+    host_tok = dev_tok = 0
+    for b, L in enumerate(lens):
+        for j in range(-(-L // 32)):
+            n = min(32, L - 32 * j)
+            if table[b, j] < res.host_split:
+                host_tok += n
+            else:
+                dev_tok += n
+    assert (res.host_tokens, res.dev_tokens) == (host_tok, dev_tok)
+    assert host_tok + dev_tok == sum(lens)
+
+
+def test_long_context_placement_numbers():
+    """1,048,576 tokens in 64-token blocks, 90% host: the oldest 14746 blocks host, newest 1638 HBM."""
+    table, res = plan([1 << 20], 64, dkv.DKV_PLACE_PREFIX_HOST, 0.9)
+    assert (res.host_split, res.num_dev_blocks) == (14746, 1638)
+    assert (table[0, :14746] < res.host_split).all() and (table[0, 14746:] >= res.host_split).all()
+
+
+def test_tiny_placement_tokens_0_255_on_host():
+    table, res = plan([512], 16, dkv.DKV_PLACE_PREFIX_HOST, 0.5)
+    assert res.host_tokens == 256 and res.dev_tokens == 256
+    assert (table[0, :16] < res.host_split).all() and (table[0, 16:] >= res.host_split).all()
+
+
+def test_extreme_fractions_and_determinism():
+    lens = [500, 800]
+    t0, r0 = plan(lens, 16, dkv.DKV_PLACE_RANDOM, 0.0, seed=5)
+    assert r0.host_split == 0
+    t1, r1 = plan(lens, 16, dkv.DKV_PLACE_RANDOM, 1.0, seed=5)
+    assert r1.num_dev_blocks == 0
+    a, _ = plan(lens, 16, dkv.DKV_PLACE_RANDOM, 0.5, True, seed=9)
+    b, _ = plan(lens, 16, dkv.DKV_PLACE_RANDOM, 0.5, True, seed=9)
+    c, _ = plan(lens, 16, dkv.DKV_PLACE_RANDOM, 0.5, True, seed=10)
+    assert np.array_equal(a, b) and not np.array_equal(a, c)
+
+
+def test_random_placement_is_roughly_uniform():
+    n = 4096
+    counts = np.zeros(n)
+    for seed in range(40):
+        table, res = plan([16 * n], 16, dkv.DKV_PLACE_RANDOM, 0.25, seed=seed)
+        counts += table[0] < res.host_split
+    # each block is on the host with probability 1/4: 40 draws -> mean 10, sd ~2.7
+    assert abs(counts.mean() - 10) < 1e-9
+    assert counts.std() < 4.0 and counts.min() >= 0 and (counts > 0).mean() > 0.95
+
+
+def test_plan_rejects_bad_arguments():
+    table = np.zeros((1, 2), dtype=np.int32)
+    with pytest.raises(dkv.DkvError):
+        dkv.dkv_plan_blocks(dkv.DkvPlanParams(16, 0, 1.5, 0, 0), np.array([10], np.int32), table)
+    with pytest.raises(dkv.DkvError):
+        dkv.dkv_plan_blocks(dkv.DkvPlanParams(16, 0, 0.5, 0, 0), np.array([100], np.int32), table)
+    with pytest.raises(dkv.DkvError):
+        dkv.dkv_plan_blocks(dkv.DkvPlanParams(16, 5, 0.5, 0, 0), np.array([10], np.int32), table)
+    with pytest.raises(dkv.DkvError):
+        dkv.dkv_plan_blocks(dkv.DkvPlanParams(16, 0, 0.5, 0, 0), np.array([-1], np.int32), table)
+
+
+@pytest.mark.parametrize("S,f,shuffle", [(16, 0.5, False), (32, 0.75, True), (64, 0.0, True), (16, 1.0, False)])
+def test_pack_places_every_token_where_the_table_says(S, f, shuffle):
+    w = kvgen.OPT_6_7B.replace(batch=3, num_q_heads=4, num_kv_heads=2, ctx=(1, 150))
+    lens = kvgen.gen_seq_lens(w)
+    k, v = kvgen.gen_kv(w, lens)
+    table, res = plan(lens, S, dkv.DKV_PLACE_RANDOM, f, shuffle, seed=2)
+    Hkv, D = w.num_kv_heads, w.head_dim
+    blk = Hkv * S * D
+    kh = np.full(max(1, res.host_split * blk), 0xFFFF, np.uint16)
+    vh = kh.copy()
+    kd = np.full(max(1, res.num_dev_blocks * blk), 0xFFFF, np.uint16)
+    vd = kd.copy()
+    dkv.dkv_pack_kv(k, v, lens, Hkv, D, S, table, res.host_split, res.num_dev_blocks, kh, vh, kd, vd)
+    for b, L in enumerate(lens):
+        for j in range(-(-int(L) // S)):
+            pid = int(table[b, j])
+            kp, vp, idx = (kh, vh, pid) if pid < res.host_split else (kd, vd, pid - res.host_split)
+            tile_k = kp[idx * blk:(idx + 1) * blk].reshape(Hkv, S, D)
+            tile_v = vp[idx * blk:(idx + 1) * blk].reshape(Hkv, S, D)
+            n = min(S, int(L) - j * S)
+            assert np.array_equal(tile_k[:, :n], k[b, :, j * S:j * S + n])
+            assert np.array_equal(tile_v[:, :n], v[b, :, j * S:j * S + n])
+            assert not tile_k[:, n:].any() and not tile_v[:, n:].any()
