@@ -35,7 +35,8 @@ DKV_PLACE_RANDOM = 1
 
 EXPORTED = ("dkv_create", "dkv_destroy", "dkv_attn_decode", "dkv_get_status", "dkv_last_error_string",
             "dkv_last_launch_count", "dkv_query_plan", "dkv_host_pool_alloc", "dkv_host_pool_free",
-            "dkv_plan_blocks", "dkv_pack_kv", "dkv_profile_begin", "dkv_profile_end")
+            "dkv_plan_blocks", "dkv_pack_kv", "dkv_profile_begin", "dkv_profile_end",
+            "dkv_attn_decode_noalloc")
 
 
 class DkvConfig(ctypes.Structure):
@@ -79,6 +80,8 @@ def _load() -> ctypes.CDLL:
         "dkv_plan_blocks": [c.POINTER(DkvPlanParams), vp, i32, vp, i32, c.POINTER(DkvPlanResult)],
         "dkv_pack_kv": [vp, vp, i64, vp, i32, i32, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp],
         "dkv_profile_begin": [vp, i32],
+        "dkv_attn_decode_noalloc": [c.POINTER(DkvConfig), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32,
+                                    i32],
         "dkv_profile_end": [vp, c.POINTER(c.c_float), c.POINTER(i32)],
     }
     for name, args in sig.items():
@@ -174,6 +177,14 @@ def dkv_pack_kv(k_logical, v_logical, seq_lens, num_kv_heads, head_dim, block_si
                            num_kv_heads, head_dim, block_size, _p(block_table), block_table.shape[1],
                            int(host_split), int(num_dev_blocks), _p(k_host), _p(v_host), _p(k_dev_stage),
                            _p(v_dev_stage)))
+
+
+def dkv_attn_decode_noalloc(cfg: DkvConfig, q, k_host, v_host, k_dev, v_dev, block_table, seq_lens, host_split,
+                            out, status_out, stream, batch, block_table_stride, num_dev_blocks) -> None:
+    """The allocation-free decode entry point (fixed scratch compiled into the library)."""
+    _check(lib.dkv_attn_decode_noalloc(ctypes.byref(cfg), _p(q), _p(k_host), _p(v_host), _p(k_dev), _p(v_dev),
+                                       _p(block_table), _p(seq_lens), int(host_split), _p(out), _p(status_out),
+                                       stream, int(batch), int(block_table_stride), int(num_dev_blocks)))
 
 
 def dkv_profile_begin(h: int, max_calls: int) -> None:

@@ -138,6 +138,41 @@ DKV_API int dkv_last_launch_count(const dkv_handle* h, int32_t* count);
 DKV_API int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_table_stride, int32_t* num_splits,
                    int32_t* blocks_per_split);
 
+/* ---- decode without any allocation ---------------------------------------
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory or keep a handle: a serving engine that
+ * hands all GPU memory to its own allocator at start-up (a library cudaMalloc
+ * would then fail or upset its accounting), a latency-critical loop in which
+ * cudaMalloc/cudaFree may synchronise the device, or a plugin behind a plain
+ * C interface that only sees raw pointers on each call.
+ *
+ * dkv_attn_decode_noalloc -- the same computation as dkv_attn_decode, with
+ * the configuration passed per call and no handle.  It allocates nothing:
+ * its scratch (status word, RoPE frequencies, split partials) is one fixed
+ * array of DKV_NOALLOC_SCRATCH_BYTES compiled into the library, held on every
+ * GPU that loads the library until the process exits.
+ *   cfg          read for this call only; cfg->max_batch is ignored, the
+ *                other fields mean what they mean for dkv_create.
+ *   status_out   device int32 or NULL: receives the DKV_STATUS_* bits of
+ *                this call (the scratch status word is cleared at its start).
+ *   other arguments as for dkv_attn_decode.  All kernels run in order on
+ *   `stream` (the host-stream and HBM kernels do not overlap here).
+ * The first call on a device looks up the device address of the scratch
+ * array (cudaGetSymbolAddress) and sets the kernels' shared-memory limits;
+ * make that first call before any stream capture.  Every call on a device
+ * shares the one array and finds the previous call's contents in it, so calls
+ * that may overlap on the GPU (other streams, other threads) race: order them.
+ * A batch whose partials cannot fit (batch * num_q_heads beyond about
+ * DKV_NOALLOC_SCRATCH_BYTES / (8 * (head_dim + 1))) is rejected with
+ * DKV_ERR_INVALID_ARG before anything is launched.  No cudaMalloc, cudaFree
+ * or other allocating call is made. */
+#define DKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const float* q, const void* k_host, const void* v_host,
+                                    const void* k_dev, const void* v_dev, const int32_t* block_table,
+                                    const int32_t* seq_lens, int32_t host_split, float* out, int32_t* status_out,
+                                    dkv_stream_t stream, int32_t batch, int32_t block_table_stride,
+                                    int32_t num_dev_blocks);
+
 /* ---- per-kernel timing ---------------------------------------------------
  * dkv_profile_begin -- record CUDA events around every kernel of the next
  * max_calls dkv_attn_decode calls, each on the stream that kernel runs on
