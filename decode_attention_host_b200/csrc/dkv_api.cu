@@ -231,6 +231,7 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   if (static_cast<long long>(c.max_blocks_per_seq) * c.block_size > (1LL << 30))
     return fail(DKV_ERR_INVALID_ARG, "max_blocks_per_seq * block_size exceeds 2^30 tokens");
   if (c.host_ctas < 0) return fail(DKV_ERR_INVALID_ARG, "host_ctas must be >= 0");
+  if (c.num_kv_heads > 4096) return fail(DKV_ERR_INVALID_ARG, "num_kv_heads must be <= 4096");
   const int G = c.num_q_heads / c.num_kv_heads;
   if (c.head_dim != 64 && c.head_dim != 128) return fail(DKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   if (G != 1 && G != 2 && G != 4) return fail(DKV_ERR_UNSUPPORTED, "query group size must be 1, 2 or 4");
@@ -333,6 +334,11 @@ int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const voi
     return fail(DKV_ERR_INVALID_ARG, "host_split / num_dev_blocks out of range");
   if (host_split > 0 && (!k_host || !v_host)) return fail(DKV_ERR_INVALID_ARG, "host pool pointers are null");
   if (num_dev_blocks > 0 && (!k_dev || !v_dev)) return fail(DKV_ERR_INVALID_ARG, "device pool pointers are null");
+  if (reinterpret_cast<uintptr_t>(q) % 8 != 0)
+    return fail(DKV_ERR_INVALID_ARG, "q must be 8-byte aligned");
+  if ((host_split > 0 && (reinterpret_cast<uintptr_t>(k_host) | reinterpret_cast<uintptr_t>(v_host)) % 16 != 0) ||
+      (num_dev_blocks > 0 && (reinterpret_cast<uintptr_t>(k_dev) | reinterpret_cast<uintptr_t>(v_dev)) % 16 != 0))
+    return fail(DKV_ERR_INVALID_ARG, "K/V pools must be 16-byte aligned");
 
   DeviceGuard guard(h->cfg.device);
   if (!guard.ok) return fail(DKV_ERR_CUDA, "cudaSetDevice failed");

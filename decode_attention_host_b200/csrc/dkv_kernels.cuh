@@ -82,7 +82,7 @@ struct TileDesc {
   int32_t unit;
   int32_t pidx;  // block index inside this pool
   int32_t p0;    // logical position of the tile's first token
-  int32_t meta;  // valid tokens (0..16) | kFlagPoison
+  int32_t meta;  // valid tokens (0..16) | kFlagPoison | kv head << 16
 };
 
 // ----------------------------------------------------------------------------- small helpers
@@ -110,35 +110,35 @@ __device__ __forceinline__ void rope_cs(int pos, double w, float& c, float& s) {
   __sincosf(static_cast<float>(r), &s, &c);
 }
 
+// Two consecutive 16-bit elements (one 32-bit word) widened to an fp32 pair.
 template <bool BF16>
-__device__ __forceinline__ void unpack2(uint32_t w, float& a, float& b) {
+__device__ __forceinline__ float2 widen2(uint32_t w) {
   if constexpr (BF16) {
-    a = __uint_as_float(w << 16);
-    b = __uint_as_float(w & 0xffff0000u);
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
   } else {
     __half2 h = *reinterpret_cast<__half2*>(&w);
-    float2 f = __half22float2(h);
-    a = f.x;
-    b = f.y;
+    return __half22float2(h);
   }
 }
 
-// PPL consecutive 16-bit elements from shared memory, widened to fp32.
-template <int PPL, bool BF16>
-__device__ __forceinline__ void load_run(const char* src, float (&x)[PPL]) {
-  if constexpr (PPL == 8) {
+// NP2 = PPL/2 fp32 pairs from PPL consecutive 16-bit elements in shared memory.
+template <int NP2, bool BF16>
+__device__ __forceinline__ void load_pairs(const char* src, float2 (&x)[NP2]) {
+  if constexpr (NP2 == 4) {
     const uint4 u = *reinterpret_cast<const uint4*>(src);
-    unpack2<BF16>(u.x, x[0], x[1]);
-    unpack2<BF16>(u.y, x[2], x[3]);
-    unpack2<BF16>(u.z, x[4], x[5]);
-    unpack2<BF16>(u.w, x[6], x[7]);
+    x[0] = widen2<BF16>(u.x);
+    x[1] = widen2<BF16>(u.y);
+    x[2] = widen2<BF16>(u.z);
+    x[3] = widen2<BF16>(u.w);
   } else {
-    static_assert(PPL == 4, "head_dim 64 or 128");
+    static_assert(NP2 == 2, "head_dim 64 or 128");
     const uint2 u = *reinterpret_cast<const uint2*>(src);
-    unpack2<BF16>(u.x, x[0], x[1]);
-    unpack2<BF16>(u.y, x[2], x[3]);
+    x[0] = widen2<BF16>(u.x);
+    x[1] = widen2<BF16>(u.y);
   }
 }
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
 // ----------------------------------------------------------------------------- tile stream
 
@@ -174,7 +174,7 @@ struct TileStream {
       if (!started) begin_unit(p);
       if (bad_len) {
         if (lane == 0) atomicOr(p.status, 2);
-        TileDesc d{unit, 0, 0, kFlagPoison};
+        TileDesc d{unit, 0, 0, kFlagPoison | (h << 16)};
         next_unit();
         return d;
       }
@@ -190,12 +190,12 @@ struct TileStream {
             if (lane == 0) atomicOr(p.status, 1);
             ++j;
             emitted = true;
-            return TileDesc{unit, 0, 0, kFlagPoison};
+            return TileDesc{unit, 0, 0, kFlagPoison | (h << 16)};
           }
         }
         const int p0 = j * p.block_size + sub * kTileTokens;
         const int nvalid = min(kTileTokens, L - p0);
-        TileDesc d{unit, pidx, p0, nvalid};
+        TileDesc d{unit, pidx, p0, nvalid | (h << 16)};
         emitted = true;
         ++sub;
         if (sub * kTileTokens >= p.block_size || p0 + kTileTokens >= L) {
@@ -207,7 +207,7 @@ struct TileStream {
       const bool was_emitted = emitted;
       const int u = unit;
       next_unit();
-      if (!was_emitted) return TileDesc{u, 0, 0, 0};  // empty unit: still reported once
+      if (!was_emitted) return TileDesc{u, 0, 0, h << 16};  // empty unit: still reported once
     }
     return TileDesc{-1, 0, 0, 0};
   }
@@ -218,11 +218,14 @@ struct TileStream {
 template <int D, int G, bool BF16, int NST>
 __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   constexpr int PPL = D / 16;                  // NeoX pairs per lane
+  constexpr int NP2 = PPL / 2;                 // fp32 pairs per half-row per lane
   constexpr int ROW = D * 2;                   // bytes of one token row
   constexpr int TILE = kTileTokens * ROW;      // bytes of one K (or V) tile
   constexpr int CPR = ROW / 16;                // 16-byte chunks per row
   extern __shared__ __align__(128) char smem[];
   __shared__ TileDesc meta[kWarps][NST];
+  __shared__ double s_freq[D / 2];             // base^(-2i/D)
+  __shared__ float2 s_step[D / 2];             // exp(i * 4 * theta_i(1)): the 4-token step
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -230,14 +233,14 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   const int li = lane & 7;
   char* ring = smem + static_cast<size_t>(warp) * NST * 2 * TILE;
 
-  // this lane's rotation frequencies and the 4-token step exp(i*4*w)
-  double w[PPL];
-  float e4c[PPL], e4s[PPL];
-#pragma unroll
-  for (int r = 0; r < PPL; ++r) {
-    w[r] = p.rope ? p.inv_freq[li * PPL + r] : 0.0;
-    rope_cs(4, w[r], e4c[r], e4s[r]);
+  for (int i = threadIdx.x; i < D / 2; i += kThreads) {
+    const double w = p.rope ? p.inv_freq[i] : 0.0;
+    float c, sn;
+    rope_cs(4, w, c, sn);
+    s_freq[i] = w;
+    s_step[i] = make_float2(c, sn);
   }
+  __syncthreads();
 
   TileStream ts;
   ts.unit = blockIdx.x * kWarps + warp;
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   auto issue = [&](const TileDesc& d, int slot) {
     const int nvalid = d.meta & 0xff;
     if (d.unit < 0 || (d.meta & kFlagPoison) || nvalid == 0) return;
-    const int h = d.unit % p.hkv;
+    const int h = d.meta >> 16;
     const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + (d.p0 % p.block_size);
     const char* gk = reinterpret_cast<const char*>(p.k_pool + row0 * D);
     const char* gv = reinterpret_cast<const char*>(p.v_pool + row0 * D);
@@ -261,34 +264,54 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     }
   };
 
-  // per-unit state
-  float qx[G][PPL], qy[G][PPL];
-  float ax[G][PPL], ay[G][PPL];
+  // per-unit state: rotated, pre-scaled queries and un-normalised outputs of
+  // this lane's dims, as fp32 pairs (first half X, second half Y)
+  float2 QX[G][NP2], QY[G][NP2];
+  float2 AX[G][NP2], AY[G][NP2];
   float mrun[G], lrun[G];
   bool poisoned = false;
   int cur = -1;
 
-  auto init_unit = [&](int unit) {
-    const int h = unit % p.hkv;
+  // cos/sin of pos * theta for this lane's pairs, as fp32 pairs
+  auto seeds = [&](int pos, float2 (&C)[NP2], float2 (&S)[NP2]) {
+#pragma unroll
+    for (int j = 0; j < NP2; ++j) {
+      float c0, s0, c1, s1;
+      rope_cs(pos, s_freq[li * PPL + 2 * j], c0, s0);
+      rope_cs(pos, s_freq[li * PPL + 2 * j + 1], c1, s1);
+      C[j] = make_float2(c0, c1);
+      S[j] = make_float2(s0, s1);
+    }
+  };
+
+  auto init_unit = [&](int unit, int h) {
     const int b = (unit / p.hkv) / p.nsplit;
     const int L = p.seq_lens[b];
-    float c[PPL], s[PPL];
+    float2 C[NP2], S[NP2];
+    if (p.rope) {
+      seeds(L, C, S);
+    } else {
 #pragma unroll
-    for (int r = 0; r < PPL; ++r) {
-      if (p.rope) rope_cs(L, w[r], c[r], s[r]);
-      else { c[r] = 1.f; s[r] = 0.f; }
+      for (int j = 0; j < NP2; ++j) {
+        C[j] = f2(1.f);
+        S[j] = f2(0.f);
+      }
     }
+    const float2 qs = f2(p.qscale);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float* qg = p.q + (static_cast<size_t>(b) * p.hq + h * G + g) * D;
 #pragma unroll
-      for (int r = 0; r < PPL; ++r) {
-        const float x = qg[li * PPL + r];
-        const float y = qg[D / 2 + li * PPL + r];
-        qx[g][r] = (x * c[r] - y * s[r]) * p.qscale;
-        qy[g][r] = (y * c[r] + x * s[r]) * p.qscale;
-        ax[g][r] = 0.f;
-        ay[g][r] = 0.f;
+      for (int j = 0; j < NP2; ++j) {
+        const float2 x = *reinterpret_cast<const float2*>(qg + li * PPL + 2 * j);
+        const float2 y = *reinterpret_cast<const float2*>(qg + D / 2 + li * PPL + 2 * j);
+        // x' = x c - y s ; y' = y c + x s, then the softmax scale (with log2 e)
+        const float2 xr = __ffma2_rn(make_float2(-y.x, -y.y), S[j], __fmul2_rn(x, C[j]));
+        const float2 yr = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));
+        QX[g][j] = __fmul2_rn(xr, qs);
+        QY[g][j] = __fmul2_rn(yr, qs);
+        AX[g][j] = f2(0.f);
+        AY[g][j] = f2(0.f);
       }
       mrun[g] = -1e30f;
       lrun[g] = 0.f;
@@ -296,8 +319,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     poisoned = false;
   };
 
-  auto finalize = [&](int unit) {
-    const int h = unit % p.hkv;
+  auto finalize = [&](int unit, int h) {
     const int bc = unit / p.hkv;
     const int c = bc % p.nsplit;
     const int b = bc / p.nsplit;
@@ -309,33 +331,35 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       float l = lrun[g] * f;
       l += __shfl_xor_sync(kFull, l, 8);
       l += __shfl_xor_sync(kFull, l, 16);
+      const float2 ff = f2(f);
 #pragma unroll
-      for (int r = 0; r < PPL; ++r) {
-        float a = ax[g][r] * f;
-        a += __shfl_xor_sync(kFull, a, 8);
-        a += __shfl_xor_sync(kFull, a, 16);
-        ax[g][r] = a;
-        float y = ay[g][r] * f;
-        y += __shfl_xor_sync(kFull, y, 8);
-        y += __shfl_xor_sync(kFull, y, 16);
-        ay[g][r] = y;
+      for (int j = 0; j < NP2; ++j) {
+        float2 a = __fmul2_rn(AX[g][j], ff);
+        a.x += __shfl_xor_sync(kFull, a.x, 8);
+        a.y += __shfl_xor_sync(kFull, a.y, 8);
+        a.x += __shfl_xor_sync(kFull, a.x, 16);
+        a.y += __shfl_xor_sync(kFull, a.y, 16);
+        AX[g][j] = a;
+        float2 y = __fmul2_rn(AY[g][j], ff);
+        y.x += __shfl_xor_sync(kFull, y.x, 8);
+        y.y += __shfl_xor_sync(kFull, y.y, 8);
+        y.x += __shfl_xor_sync(kFull, y.x, 16);
+        y.y += __shfl_xor_sync(kFull, y.y, 16);
+        AY[g][j] = y;
       }
       if (tg == 0) {
         const size_t row = (static_cast<size_t>(b) * p.hq + h * G + g) * p.nslots + p.slot_base + c;
         float* o = p.part_o + row * D;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float qnan = __int_as_float(0x7fc00000);
+        const float2 inv = f2(poisoned ? qnan : (l > 0.f ? 1.f / l : 0.f));
         float lse = l > 0.f ? M + __log2f(l) : -INFINITY;
-        float ox[PPL], oy[PPL];
+        if (poisoned) lse = qnan;
 #pragma unroll
-        for (int r = 0; r < PPL; ++r) {
-          ox[r] = poisoned ? __int_as_float(0x7fc00000) : ax[g][r] * inv;
-          oy[r] = poisoned ? __int_as_float(0x7fc00000) : ay[g][r] * inv;
-        }
-        if (poisoned) lse = __int_as_float(0x7fc00000);
-#pragma unroll
-        for (int r = 0; r < PPL; r += 4) {
-          *reinterpret_cast<float4*>(o + li * PPL + r) = make_float4(ox[r], ox[r + 1], ox[r + 2], ox[r + 3]);
-          *reinterpret_cast<float4*>(o + D / 2 + li * PPL + r) = make_float4(oy[r], oy[r + 1], oy[r + 2], oy[r + 3]);
+        for (int j = 0; j < NP2; j += 2) {
+          const float2 x0 = __fmul2_rn(AX[g][j], inv), x1 = __fmul2_rn(AX[g][j + 1], inv);
+          const float2 y0 = __fmul2_rn(AY[g][j], inv), y1 = __fmul2_rn(AY[g][j + 1], inv);
+          *reinterpret_cast<float4*>(o + li * PPL + 2 * j) = make_float4(x0.x, x0.y, x1.x, x1.y);
+          *reinterpret_cast<float4*>(o + D / 2 + li * PPL + 2 * j) = make_float4(y0.x, y0.y, y1.x, y1.y);
         }
         if (li == 0) p.part_lse[row] = lse;
       }
@@ -346,37 +370,46 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const char* sk = ring + static_cast<size_t>(slot) * 2 * TILE;
     const char* sv = sk + TILE;
     const int nvalid = d.meta & 0xff;
-    float c[PPL], s[PPL];
+    float2 C[NP2], S[NP2], E[NP2], F[NP2];
+    if (p.rope) {
+      seeds(d.p0 + tg, C, S);
 #pragma unroll
-    for (int r = 0; r < PPL; ++r) {
-      if (p.rope) rope_cs(d.p0 + tg, w[r], c[r], s[r]);
-      else { c[r] = 1.f; s[r] = 0.f; }
+      for (int j = 0; j < NP2; ++j) {
+        const float2 a = s_step[li * PPL + 2 * j], b = s_step[li * PPL + 2 * j + 1];
+        E[j] = make_float2(a.x, b.x);
+        F[j] = make_float2(a.y, b.y);
+      }
     }
     float sc[4][G];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const char* row = sk + (tg + 4 * m) * ROW;
-      float kx[PPL], ky[PPL];
-      load_run<PPL, BF16>(row + li * PPL * 2, kx);
-      load_run<PPL, BF16>(row + D + li * PPL * 2, ky);
+      float2 X[NP2], Y[NP2];
+      load_pairs<NP2, BF16>(row + li * PPL * 2, X);
+      load_pairs<NP2, BF16>(row + D + li * PPL * 2, Y);
+      if (p.rope) {
 #pragma unroll
-      for (int r = 0; r < PPL; ++r) {
-        const float x = kx[r], y = ky[r];
-        kx[r] = x * c[r] - y * s[r];
-        ky[r] = y * c[r] + x * s[r];
-        const float cn = c[r] * e4c[r] - s[r] * e4s[r];
-        s[r] = s[r] * e4c[r] + c[r] * e4s[r];
-        c[r] = cn;
+        for (int j = 0; j < NP2; ++j) {
+          const float2 x = X[j], y = Y[j];
+          X[j] = __ffma2_rn(make_float2(-y.x, -y.y), S[j], __fmul2_rn(x, C[j]));
+          Y[j] = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));
+          if (m < 3) {  // advance 4 positions: (C + iS)(E + iF)
+            const float2 cn = __ffma2_rn(make_float2(-S[j].x, -S[j].y), F[j], __fmul2_rn(C[j], E[j]));
+            S[j] = __ffma2_rn(C[j], F[j], __fmul2_rn(S[j], E[j]));
+            C[j] = cn;
+          }
+        }
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float a = 0.f;
+        float2 a = __fmul2_rn(QX[g][0], X[0]);
+        a = __ffma2_rn(QY[g][0], Y[0], a);
 #pragma unroll
-        for (int r = 0; r < PPL; ++r) {
-          a = fmaf(qx[g][r], kx[r], a);
-          a = fmaf(qy[g][r], ky[r], a);
+        for (int j = 1; j < NP2; ++j) {
+          a = __ffma2_rn(QX[g][j], X[j], a);
+          a = __ffma2_rn(QY[g][j], Y[j], a);
         }
-        sc[m][g] = a;
+        sc[m][g] = a.x + a.y;
       }
     }
 #pragma unroll
@@ -404,26 +437,29 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       lrun[g] = lrun[g] * alpha + sum;
       mrun[g] = mx;
       if (alpha != 1.f) {
+        const float2 al = f2(alpha);
 #pragma unroll
-        for (int r = 0; r < PPL; ++r) {
-          ax[g][r] *= alpha;
-          ay[g][r] *= alpha;
+        for (int j = 0; j < NP2; ++j) {
+          AX[g][j] = __fmul2_rn(AX[g][j], al);
+          AY[g][j] = __fmul2_rn(AY[g][j], al);
         }
       }
     }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const char* row = sv + (tg + 4 * m) * ROW;
-      float vx[PPL], vy[PPL];
-      load_run<PPL, BF16>(row + li * PPL * 2, vx);
-      load_run<PPL, BF16>(row + D + li * PPL * 2, vy);
+      float2 X[NP2], Y[NP2];
+      load_pairs<NP2, BF16>(row + li * PPL * 2, X);
+      load_pairs<NP2, BF16>(row + D + li * PPL * 2, Y);
 #pragma unroll
-      for (int g = 0; g < G; ++g)
+      for (int g = 0; g < G; ++g) {
+        const float2 pp = f2(pr[m][g]);
 #pragma unroll
-        for (int r = 0; r < PPL; ++r) {
-          ax[g][r] = fmaf(pr[m][g], vx[r], ax[g][r]);
-          ay[g][r] = fmaf(pr[m][g], vy[r], ay[g][r]);
+        for (int j = 0; j < NP2; ++j) {
+          AX[g][j] = __ffma2_rn(pp, X[j], AX[g][j]);
+          AY[g][j] = __ffma2_rn(pp, Y[j], AY[g][j]);
         }
+      }
     }
   };
 
@@ -435,6 +471,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     issue(d, s);
     cp_async_commit();
   }
+  int cur_h = 0;
 #pragma unroll 1
   for (int k = 0;; ++k) {
     {
@@ -450,15 +487,16 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const TileDesc d = meta[warp][slot];
     if (d.unit < 0) break;
     if (d.unit != cur) {
-      if (cur >= 0) finalize(cur);
-      init_unit(d.unit);
+      if (cur >= 0) finalize(cur, cur_h);
       cur = d.unit;
+      cur_h = d.meta >> 16;
+      init_unit(cur, cur_h);
     }
     if (d.meta & kFlagPoison) poisoned = true;
     else if ((d.meta & 0xff) > 0) compute(slot, d);
     __syncwarp();
   }
-  if (cur >= 0) finalize(cur);
+  if (cur >= 0) finalize(cur, cur_h);
   cp_async_wait<0>();
 }
 

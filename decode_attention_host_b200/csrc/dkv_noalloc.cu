@@ -130,7 +130,7 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
   using dkv::set_error;
   if (!cfg) return set_error(DKV_ERR_INVALID_ARG, "dkv_attn_decode_noalloc: null config");
   const dkv_config& c = *cfg;
-  if (c.num_q_heads < 1 || c.num_kv_heads < 1 || c.num_q_heads % c.num_kv_heads != 0 || c.block_size < 16 ||
+  if (c.num_q_heads < 1 || c.num_kv_heads < 1 || c.num_kv_heads > 4096 || c.num_q_heads % c.num_kv_heads != 0 || c.block_size < 16 ||
       c.block_size > 1024 || c.block_size % 16 != 0 || (c.kv_dtype != DKV_KV_F16 && c.kv_dtype != DKV_KV_BF16) ||
       !(c.rope_base >= 0.0) || !(c.rope_base < 1e300) || (c.rope_base > 0.0 && c.rope_base <= 1.0) ||
       !(c.scale >= 0.0) || !(c.scale < 1e300) || c.max_blocks_per_seq < 1 ||
@@ -146,6 +146,10 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
       static_cast<long long>(host_split) + num_dev_blocks > 0x7fffffffLL || (host_split > 0 && (!k_host || !v_host)) ||
       (num_dev_blocks > 0 && (!k_dev || !v_dev)))
     return set_error(DKV_ERR_INVALID_ARG, "dkv_attn_decode_noalloc: null pointer or size out of range");
+  if (reinterpret_cast<uintptr_t>(q) % 8 != 0 ||
+      (host_split > 0 && (reinterpret_cast<uintptr_t>(k_host) | reinterpret_cast<uintptr_t>(v_host)) % 16 != 0) ||
+      (num_dev_blocks > 0 && (reinterpret_cast<uintptr_t>(k_dev) | reinterpret_cast<uintptr_t>(v_dev)) % 16 != 0))
+    return set_error(DKV_ERR_INVALID_ARG, "dkv_attn_decode_noalloc: q must be 8-byte and pools 16-byte aligned");
   const int D = c.head_dim;
   // even one split per side must fit in the fixed scratch array
   const size_t min_rows = static_cast<size_t>(batch) * c.num_q_heads * 2;

@@ -58,7 +58,7 @@ typedef enum { DKV_KV_F16 = 0, DKV_KV_BF16 = 1 } dkv_kv_dtype;
 
 typedef struct dkv_config {
   int32_t num_q_heads;        /* Hq >= 1 */
-  int32_t num_kv_heads;       /* Hkv >= 1, Hq % Hkv == 0; G = Hq/Hkv in {1, 2, 4} */
+  int32_t num_kv_heads;       /* 1 <= Hkv <= 4096, Hq % Hkv == 0; G = Hq/Hkv in {1, 2, 4} */
   int32_t head_dim;           /* D in {64, 128} */
   int32_t block_size;         /* S tokens per block: multiple of 16, 16 <= S <= 1024 */
   int32_t kv_dtype;           /* dkv_kv_dtype */
@@ -90,7 +90,8 @@ DKV_API int dkv_destroy(dkv_handle* h);
 /*
  * dkv_attn_decode -- one decode-attention step for a batch of sequences.
  *
- *   q            device, fp32 [batch][Hq][D]: the new token's query, un-rotated.
+ *   q            device, fp32 [batch][Hq][D]: the new token's query, un-rotated;
+ *                8-byte aligned.  All four pool pointers must be 16-byte aligned.
  *   k_host,v_host  device aliases of MAPPED pinned host memory (see
  *                dkv_host_pool_alloc), pool layout, >= host_split blocks.
  *                May be NULL only when host_split == 0.

@@ -164,7 +164,9 @@ def test_host_side_argument_errors():
                 stream=torch.cuda.current_stream().cuda_stream, batch=1, block_table_stride=kv.stride,
                 num_dev_blocks=kv.num_dev_blocks)
     bad = [dict(k_host=pageable), dict(k_host=kv.k_dev.data_ptr()), dict(k_dev=kv.k_host.ptr), dict(batch=2),
-           dict(block_table_stride=0), dict(host_split=-1), dict(q=None), dict(k_dev=None)]
+           dict(block_table_stride=0), dict(host_split=-1), dict(q=None), dict(k_dev=None),
+           dict(q=case.q_dev.data_ptr() + 4), dict(k_dev=kv.k_dev.data_ptr() + 2),
+           dict(v_host=kv.v_host.ptr + 8)]
     for override in bad:
         a = dict(args, **override)
         with pytest.raises(dkv.DkvError) as e:
