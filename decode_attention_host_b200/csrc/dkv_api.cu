@@ -61,13 +61,13 @@ size_t split_smem(int D, int nst) { return static_cast<size_t>(dkv::kWarps) * ns
 using SplitFn = void (*)(dim3, size_t, cudaStream_t, const dkv::SplitParams&);
 using SplitKernelPtr = const void*;
 
-template <int D, int G, bool BF16, int NST>
+template <int D, int G, bool BF16, int NST, bool ROPE>
 void launch_split(dim3 grid, size_t smem, cudaStream_t s, const dkv::SplitParams& p) {
-  dkv::split_kernel<D, G, BF16, NST><<<grid, dkv::kThreads, smem, s>>>(p);
+  dkv::split_kernel<D, G, BF16, NST, ROPE><<<grid, dkv::kThreads, smem, s>>>(p);
 }
-template <int D, int G, bool BF16, int NST>
+template <int D, int G, bool BF16, int NST, bool ROPE>
 const void* split_ptr() {
-  return reinterpret_cast<const void*>(&dkv::split_kernel<D, G, BF16, NST>);
+  return reinterpret_cast<const void*>(&dkv::split_kernel<D, G, BF16, NST, ROPE>);
 }
 
 struct SplitEntry {
@@ -75,12 +75,12 @@ struct SplitEntry {
   SplitKernelPtr ptr;
 };
 
-template <int NST>
-SplitEntry pick_split(int D, int G, bool bf16) {
-#define DKV_CASE(DD, GG)                                                                   \
-  if (D == DD && G == GG) {                                                                \
-    if (bf16) return {&launch_split<DD, GG, true, NST>, split_ptr<DD, GG, true, NST>()};   \
-    return {&launch_split<DD, GG, false, NST>, split_ptr<DD, GG, false, NST>()};           \
+template <int NST, bool ROPE>
+SplitEntry pick_split_rope(int D, int G, bool bf16) {
+#define DKV_CASE(DD, GG)                                                                                   \
+  if (D == DD && G == GG) {                                                                                \
+    if (bf16) return {&launch_split<DD, GG, true, NST, ROPE>, split_ptr<DD, GG, true, NST, ROPE>()};      \
+    return {&launch_split<DD, GG, false, NST, ROPE>, split_ptr<DD, GG, false, NST, ROPE>()};              \
   }
   DKV_CASE(64, 1)
   DKV_CASE(64, 2)
@@ -90,6 +90,11 @@ SplitEntry pick_split(int D, int G, bool bf16) {
   DKV_CASE(128, 4)
 #undef DKV_CASE
   return {nullptr, nullptr};
+}
+
+template <int NST>
+SplitEntry pick_split(int D, int G, bool bf16, bool rope) {
+  return rope ? pick_split_rope<NST, true>(D, G, bf16) : pick_split_rope<NST, false>(D, G, bf16);
 }
 
 using MergeFn = void (*)(dim3, size_t, cudaStream_t, const dkv::MergeParams&);
@@ -249,8 +254,9 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   const double scale = c.scale > 0.0 ? c.scale : 1.0 / std::sqrt(static_cast<double>(c.head_dim));
   h->qscale = static_cast<float>(scale * 1.4426950408889634);  // * log2(e)
   h->host_ctas = c.host_ctas > 0 ? c.host_ctas : kDefaultHostCtas;
-  h->host_kernel = pick_split<kHostStages>(c.head_dim, G, bf16);
-  h->dev_kernel = pick_split<kDevStages>(c.head_dim, G, bf16);
+  const bool rope = c.rope_base > 0.0;
+  h->host_kernel = pick_split<kHostStages>(c.head_dim, G, bf16, rope);
+  h->dev_kernel = pick_split<kDevStages>(c.head_dim, G, bf16, rope);
   h->merge = c.head_dim == 64 ? &launch_merge<64, 4> : &launch_merge<128, 2>;
 
   auto bail = [&](int code) {

@@ -39,6 +39,7 @@
 // softmax works with exp2.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -140,6 +141,62 @@ __device__ __forceinline__ void load_pairs(const char* src, float2 (&x)[NP2]) {
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
+// 2^x in one MUFU op (flushes subnormal results to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Byte offset of 16-byte chunk c of row r in a tile of ROW-byte rows.  The
+// chunk index is XORed with the row (mod 8), so the 8 rows read by one
+// ldmatrix phase, and the 8 lanes of one token row, hit 8 distinct bank groups.
+template <int ROW>
+__device__ __forceinline__ int swz(int r, int c) {
+  return r * ROW + ((c ^ (r & 7)) << 4);
+}
+
+// Four 8x8 b16 matrices from shared memory, transposed (mma B operand).
+__device__ __forceinline__ void ldsm_x4_t(const void* p, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
+}
+
+// D(16x8,f32) += A(16x16) * B(16x8), A and B both bf16 or both fp16.
+template <bool BF16>
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (BF16) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};\n"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};\n"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+// p ~= hi + lo with hi, lo in the 16-bit type of V: returns packed hi pair and lo pair.
+template <bool BF16>
+__device__ __forceinline__ void split_hi_lo(float2 p, uint32_t& hi, uint32_t& lo) {
+  if constexpr (BF16) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(p.x, p.y);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(p.x - hf.x, p.y - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+  } else {
+    const __half2 h = __floats2half2_rn(p.x, p.y);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(p.x - hf.x, p.y - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+  }
+}
+
 // ----------------------------------------------------------------------------- tile stream
 
 // Enumerates, for one warp, the tiles of this residency over its units.  All
@@ -215,30 +272,41 @@ struct TileStream {
 
 // ----------------------------------------------------------------------------- split kernel
 
-template <int D, int G, bool BF16, int NST>
+template <int D, int G, bool BF16, int NST, bool ROPE>
 __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
+  static_assert(G >= 1 && G <= 4, "query group of 1, 2 or 4 heads");
   constexpr int PPL = D / 16;                  // NeoX pairs per lane
   constexpr int NP2 = PPL / 2;                 // fp32 pairs per half-row per lane
   constexpr int ROW = D * 2;                   // bytes of one token row
   constexpr int TILE = kTileTokens * ROW;      // bytes of one K (or V) tile
   constexpr int CPR = ROW / 16;                // 16-byte chunks per row
+  constexpr int NT = D / 8;                    // 8-wide output column tiles of the PV mma
   extern __shared__ __align__(128) char smem[];
   __shared__ TileDesc meta[kWarps][NST];
-  __shared__ double s_freq[D / 2];             // base^(-2i/D)
-  __shared__ float2 s_step[D / 2];             // exp(i * 4 * theta_i(1)): the 4-token step
+  __shared__ double s_freq[PPL][8];            // [r][li]: base^(-2i/D), i = li*PPL + r
+  __shared__ float2 s_e[NP2][8], s_f[NP2][8], s_nf[NP2][8];  // 4-token step: cos, sin, -sin (pairs)
+  __shared__ __align__(16) float s_p[kWarps][4][4][4];  // softmax weights of the tile: [head][token group][m]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int tg = lane >> 3;
-  const int li = lane & 7;
+  const int tg = lane >> 3;                    // token group (K side)
+  const int li = lane & 7;                     // lane in token group
+  const int gT = lane >> 2;                    // head row of the mma fragments
+  const int cT = lane & 3;                     // column pair of the mma fragments
   char* ring = smem + static_cast<size_t>(warp) * NST * 2 * TILE;
 
   for (int i = threadIdx.x; i < D / 2; i += kThreads) {
-    const double w = p.rope ? p.inv_freq[i] : 0.0;
+    const double w = ROPE ? p.inv_freq[i] : 0.0;
+    const int l = i / PPL, r = i % PPL;
+    s_freq[r][l] = w;
     float c, sn;
     rope_cs(4, w, c, sn);
-    s_freq[i] = w;
-    s_step[i] = make_float2(c, sn);
+    float* e = reinterpret_cast<float*>(&s_e[r >> 1][l]) + (r & 1);
+    float* f = reinterpret_cast<float*>(&s_f[r >> 1][l]) + (r & 1);
+    float* nf = reinterpret_cast<float*>(&s_nf[r >> 1][l]) + (r & 1);
+    *e = c;
+    *f = sn;
+    *nf = -sn;
   }
   __syncthreads();
 
@@ -247,38 +315,58 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   ts.unit_stride = gridDim.x * kWarps;
   ts.started = false;
 
+  // Copy chunk e = lane + 32 k of a tile: K rows are stored as they come; V rows
+  // have their 16-byte chunks XOR-swizzled by (row mod 8) so that ldmatrix,
+  // which reads one chunk column of 8 rows, touches 8 distinct bank groups.
+  // For ROW = 256 the swizzled offsets repeat every 4 copies (plus 2 KB).
+  constexpr int KCOPIES = kTileTokens * CPR / 32;
+  int vofs[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int e = lane + 32 * k;
+    vofs[k] = swz<ROW>(e / CPR, e % CPR);
+  }
   auto issue = [&](const TileDesc& d, int slot) {
     const int nvalid = d.meta & 0xff;
     if (d.unit < 0 || (d.meta & kFlagPoison) || nvalid == 0) return;
     const int h = d.meta >> 16;
     const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + (d.p0 % p.block_size);
-    const char* gk = reinterpret_cast<const char*>(p.k_pool + row0 * D);
-    const char* gv = reinterpret_cast<const char*>(p.v_pool + row0 * D);
-    char* sk = ring + static_cast<size_t>(slot) * 2 * TILE;
-    char* sv = sk + TILE;
+    const char* gk = reinterpret_cast<const char*>(p.k_pool + row0 * D) + lane * 16;
+    const char* gv = reinterpret_cast<const char*>(p.v_pool + row0 * D) + lane * 16;
+    char* sk = ring + static_cast<size_t>(slot) * 2 * TILE + lane * 16;
+    char* sv = ring + static_cast<size_t>(slot) * 2 * TILE + TILE;
+    if (nvalid == kTileTokens) {
 #pragma unroll
-    for (int e = lane; e < kTileTokens * CPR; e += 32) {
-      const int nb = (e / CPR) < nvalid ? 16 : 0;
-      cp_async16(sk + e * 16, nb ? gk + e * 16 : gk, nb);
-      cp_async16(sv + e * 16, nb ? gv + e * 16 : gv, nb);
+      for (int k = 0; k < KCOPIES; ++k) {
+        cp_async16(sk + 512 * k, gk + 512 * k, 16);
+        cp_async16(sv + vofs[k & 3] + (k >> 2) * 2048, gv + 512 * k, 16);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < KCOPIES; ++k) {
+        const int r = (lane + 32 * k) / CPR;
+        const int nb = r < nvalid ? 16 : 0;
+        cp_async16(sk + 512 * k, nb ? gk + 512 * k : gk - lane * 16, nb);
+        cp_async16(sv + vofs[k & 3] + (k >> 2) * 2048, nb ? gv + 512 * k : gv - lane * 16, nb);
+      }
     }
   };
 
-  // per-unit state: rotated, pre-scaled queries and un-normalised outputs of
-  // this lane's dims, as fp32 pairs (first half X, second half Y)
+  // per-unit state.  QX/QY: rotated, pre-scaled queries of this lane's dims.
+  // acc: PV accumulators in mma C layout -- rows 0..G-1 hold the bf16/fp16 "hi"
+  // part of the weights, rows 8..8+G-1 the "lo" remainder; out = row g + row g+8.
   float2 QX[G][NP2], QY[G][NP2];
-  float2 AX[G][NP2], AY[G][NP2];
+  float acc[NT][4];
   float mrun[G], lrun[G];
   bool poisoned = false;
   int cur = -1;
 
-  // cos/sin of pos * theta for this lane's pairs, as fp32 pairs
   auto seeds = [&](int pos, float2 (&C)[NP2], float2 (&S)[NP2]) {
 #pragma unroll
     for (int j = 0; j < NP2; ++j) {
       float c0, s0, c1, s1;
-      rope_cs(pos, s_freq[li * PPL + 2 * j], c0, s0);
-      rope_cs(pos, s_freq[li * PPL + 2 * j + 1], c1, s1);
+      rope_cs(pos, s_freq[2 * j][li], c0, s0);
+      rope_cs(pos, s_freq[2 * j + 1][li], c1, s1);
       C[j] = make_float2(c0, c1);
       S[j] = make_float2(s0, s1);
     }
@@ -288,7 +376,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const int b = (unit / p.hkv) / p.nsplit;
     const int L = p.seq_lens[b];
     float2 C[NP2], S[NP2];
-    if (p.rope) {
+    if constexpr (ROPE) {
       seeds(L, C, S);
     } else {
 #pragma unroll
@@ -305,17 +393,17 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       for (int j = 0; j < NP2; ++j) {
         const float2 x = *reinterpret_cast<const float2*>(qg + li * PPL + 2 * j);
         const float2 y = *reinterpret_cast<const float2*>(qg + D / 2 + li * PPL + 2 * j);
-        // x' = x c - y s ; y' = y c + x s, then the softmax scale (with log2 e)
-        const float2 xr = __ffma2_rn(make_float2(-y.x, -y.y), S[j], __fmul2_rn(x, C[j]));
-        const float2 yr = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));
-        QX[g][j] = __fmul2_rn(xr, qs);
-        QY[g][j] = __fmul2_rn(yr, qs);
-        AX[g][j] = f2(0.f);
-        AY[g][j] = f2(0.f);
+        const float2 xr = __fmul2_rn(x, C[j]);
+        const float2 yr = __fmul2_rn(y, C[j]);
+        const float2 ys = __fmul2_rn(y, S[j]);
+        QX[g][j] = __fmul2_rn(make_float2(xr.x - ys.x, xr.y - ys.y), qs);   // x c - y s
+        QY[g][j] = __fmul2_rn(__ffma2_rn(x, S[j], yr), qs);                  // y c + x s
       }
       mrun[g] = -1e30f;
       lrun[g] = 0.f;
     }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
     poisoned = false;
   };
 
@@ -323,46 +411,28 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const int bc = unit / p.hkv;
     const int c = bc % p.nsplit;
     const int b = bc / p.nsplit;
+    float ltot[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float M = fmaxf(mrun[g], __shfl_xor_sync(kFull, mrun[g], 8));
-      M = fmaxf(M, __shfl_xor_sync(kFull, M, 16));
-      const float f = exp2f(mrun[g] - M);
-      float l = lrun[g] * f;
+      float l = lrun[g];
       l += __shfl_xor_sync(kFull, l, 8);
       l += __shfl_xor_sync(kFull, l, 16);
-      const float2 ff = f2(f);
+      ltot[g] = l;
+    }
+    if (gT < G) {
+      float l = ltot[0], M = mrun[0];
 #pragma unroll
-      for (int j = 0; j < NP2; ++j) {
-        float2 a = __fmul2_rn(AX[g][j], ff);
-        a.x += __shfl_xor_sync(kFull, a.x, 8);
-        a.y += __shfl_xor_sync(kFull, a.y, 8);
-        a.x += __shfl_xor_sync(kFull, a.x, 16);
-        a.y += __shfl_xor_sync(kFull, a.y, 16);
-        AX[g][j] = a;
-        float2 y = __fmul2_rn(AY[g][j], ff);
-        y.x += __shfl_xor_sync(kFull, y.x, 8);
-        y.y += __shfl_xor_sync(kFull, y.y, 8);
-        y.x += __shfl_xor_sync(kFull, y.x, 16);
-        y.y += __shfl_xor_sync(kFull, y.y, 16);
-        AY[g][j] = y;
-      }
-      if (tg == 0) {
-        const size_t row = (static_cast<size_t>(b) * p.hq + h * G + g) * p.nslots + p.slot_base + c;
-        float* o = p.part_o + row * D;
-        const float qnan = __int_as_float(0x7fc00000);
-        const float2 inv = f2(poisoned ? qnan : (l > 0.f ? 1.f / l : 0.f));
-        float lse = l > 0.f ? M + __log2f(l) : -INFINITY;
-        if (poisoned) lse = qnan;
+      for (int g = 1; g < G; ++g)
+        if (gT == g) { l = ltot[g]; M = mrun[g]; }
+      const size_t row = (static_cast<size_t>(b) * p.hq + h * G + gT) * p.nslots + p.slot_base + c;
+      float* o = p.part_o + row * D;
+      const float qnan = __int_as_float(0x7fc00000);
+      const float inv = poisoned ? qnan : (l > 0.f ? 1.f / l : 0.f);
 #pragma unroll
-        for (int j = 0; j < NP2; j += 2) {
-          const float2 x0 = __fmul2_rn(AX[g][j], inv), x1 = __fmul2_rn(AX[g][j + 1], inv);
-          const float2 y0 = __fmul2_rn(AY[g][j], inv), y1 = __fmul2_rn(AY[g][j + 1], inv);
-          *reinterpret_cast<float4*>(o + li * PPL + 2 * j) = make_float4(x0.x, x0.y, x1.x, x1.y);
-          *reinterpret_cast<float4*>(o + D / 2 + li * PPL + 2 * j) = make_float4(y0.x, y0.y, y1.x, y1.y);
-        }
-        if (li == 0) p.part_lse[row] = lse;
-      }
+      for (int n = 0; n < NT; ++n)
+        *reinterpret_cast<float2*>(o + 8 * n + 2 * cT) =
+            make_float2((acc[n][0] + acc[n][2]) * inv, (acc[n][1] + acc[n][3]) * inv);
+      if (cT == 0) p.part_lse[row] = poisoned ? qnan : (l > 0.f ? M + __log2f(l) : -INFINITY);
     }
   };
 
@@ -370,33 +440,34 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const char* sk = ring + static_cast<size_t>(slot) * 2 * TILE;
     const char* sv = sk + TILE;
     const int nvalid = d.meta & 0xff;
-    float2 C[NP2], S[NP2], E[NP2], F[NP2];
-    if (p.rope) {
+    // ---- scores: rotate K rows on the fly (CUDA cores, fp32 pairs)
+    float2 C[NP2], S[NP2], NS[NP2];
+    if constexpr (ROPE) {
       seeds(d.p0 + tg, C, S);
 #pragma unroll
-      for (int j = 0; j < NP2; ++j) {
-        const float2 a = s_step[li * PPL + 2 * j], b = s_step[li * PPL + 2 * j + 1];
-        E[j] = make_float2(a.x, b.x);
-        F[j] = make_float2(a.y, b.y);
-      }
+      for (int j = 0; j < NP2; ++j) NS[j] = make_float2(-S[j].x, -S[j].y);
     }
     float sc[4][G];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const char* row = sk + (tg + 4 * m) * ROW;
+      const int t = tg + 4 * m;
       float2 X[NP2], Y[NP2];
-      load_pairs<NP2, BF16>(row + li * PPL * 2, X);
-      load_pairs<NP2, BF16>(row + D + li * PPL * 2, Y);
-      if (p.rope) {
+      const char* krow = sk + t * ROW + li * PPL * 2;
+      load_pairs<NP2, BF16>(krow, X);
+      load_pairs<NP2, BF16>(krow + D, Y);
+      if constexpr (ROPE) {
 #pragma unroll
         for (int j = 0; j < NP2; ++j) {
           const float2 x = X[j], y = Y[j];
-          X[j] = __ffma2_rn(make_float2(-y.x, -y.y), S[j], __fmul2_rn(x, C[j]));
-          Y[j] = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));
+          X[j] = __ffma2_rn(y, NS[j], __fmul2_rn(x, C[j]));   // x c - y s
+          Y[j] = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));    // y c + x s
           if (m < 3) {  // advance 4 positions: (C + iS)(E + iF)
-            const float2 cn = __ffma2_rn(make_float2(-S[j].x, -S[j].y), F[j], __fmul2_rn(C[j], E[j]));
-            S[j] = __ffma2_rn(C[j], F[j], __fmul2_rn(S[j], E[j]));
+            const float2 e = s_e[j][li], f = s_f[j][li], nf = s_nf[j][li];
+            const float2 cn = __ffma2_rn(NS[j], f, __fmul2_rn(C[j], e));
+            const float2 sn = __ffma2_rn(C[j], f, __fmul2_rn(S[j], e));
+            NS[j] = __ffma2_rn(C[j], nf, __fmul2_rn(NS[j], e));
             C[j] = cn;
+            S[j] = sn;
           }
         }
       }
@@ -422,44 +493,54 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
         a += __shfl_xor_sync(kFull, a, 4);
         sc[m][g] = (tg + 4 * m) < nvalid ? a : -INFINITY;
       }
-    float pr[4][G];
+    // ---- online softmax, one running max per head for the whole warp
+    float alpha[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float mx = fmaxf(fmaxf(sc[0][g], sc[1][g]), fmaxf(sc[2][g], sc[3][g]));
-      mx = fmaxf(mx, mrun[g]);
-      const float alpha = exp2f(mrun[g] - mx);
-      float sum = 0.f;
+      float tm = fmaxf(fmaxf(sc[0][g], sc[1][g]), fmaxf(sc[2][g], sc[3][g]));
+      tm = fmaxf(tm, __shfl_xor_sync(kFull, tm, 8));
+      tm = fmaxf(tm, __shfl_xor_sync(kFull, tm, 16));
+      const float mx = fmaxf(mrun[g], tm);
+      alpha[g] = ex2(mrun[g] - mx);
+      float pv[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        pr[m][g] = exp2f(sc[m][g] - mx);
-        sum += pr[m][g];
-      }
-      lrun[g] = lrun[g] * alpha + sum;
+      for (int m = 0; m < 4; ++m) pv[m] = ex2(sc[m][g] - mx);
+      if (li == 0) *reinterpret_cast<float4*>(&s_p[warp][g][tg][0]) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+      lrun[g] = lrun[g] * alpha[g] + ((pv[0] + pv[1]) + (pv[2] + pv[3]));
       mrun[g] = mx;
-      if (alpha != 1.f) {
-        const float2 al = f2(alpha);
+    }
+    __syncwarp();
+    // ---- PV on the tensor cores: A = weights (hi rows 0..G-1, lo rows 8..), B = V
+    uint32_t a[4] = {0u, 0u, 0u, 0u};
+    float al = 1.f;
+    if (gT < G) {
 #pragma unroll
-        for (int j = 0; j < NP2; ++j) {
-          AX[g][j] = __fmul2_rn(AX[g][j], al);
-          AY[g][j] = __fmul2_rn(AY[g][j], al);
-        }
+      for (int g = 0; g < G; ++g)
+        if (gT == g) al = alpha[g];
+      // tokens 2c, 2c+1 (a) and 2c+8, 2c+9 (b); token t lives at [t % 4][t / 4]
+      const float* sp = &s_p[warp][gT][0][0];
+      const int t0 = 2 * cT;
+      const float2 pa = make_float2(sp[(t0 & 3) * 4 + (t0 >> 2)], sp[((t0 + 1) & 3) * 4 + (t0 >> 2)]);
+      const float2 pb = make_float2(sp[(t0 & 3) * 4 + (t0 >> 2) + 2], sp[((t0 + 1) & 3) * 4 + (t0 >> 2) + 2]);
+      split_hi_lo<BF16>(pa, a[0], a[1]);
+      split_hi_lo<BF16>(pb, a[2], a[3]);
+    }
+    if (al != 1.f) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        acc[n][0] *= al;
+        acc[n][1] *= al;
+        acc[n][2] *= al;
+        acc[n][3] *= al;
       }
     }
+    const int vrow = (lane & 7) | (lane & 8);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const char* row = sv + (tg + 4 * m) * ROW;
-      float2 X[NP2], Y[NP2];
-      load_pairs<NP2, BF16>(row + li * PPL * 2, X);
-      load_pairs<NP2, BF16>(row + D + li * PPL * 2, Y);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float2 pp = f2(pr[m][g]);
-#pragma unroll
-        for (int j = 0; j < NP2; ++j) {
-          AX[g][j] = __ffma2_rn(pp, X[j], AX[g][j]);
-          AY[g][j] = __ffma2_rn(pp, Y[j], AY[g][j]);
-        }
-      }
+    for (int qd = 0; qd < D / 16; ++qd) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(sv + swz<ROW>(vrow, 2 * qd + (lane >> 4)), b0, b1, b2, b3);
+      mma16816<BF16>(acc[2 * qd], a, b0, b1);
+      mma16816<BF16>(acc[2 * qd + 1], a, b2, b3);
     }
   };
 

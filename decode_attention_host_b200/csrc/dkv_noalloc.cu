@@ -58,19 +58,19 @@ struct SplitVariant {
   const void* fn;
 };
 
-template <int D, int G, bool BF16, int NST>
+template <int D, int G, bool BF16, int NST, bool ROPE>
 void launch_split(dim3 grid, size_t smem, cudaStream_t s, const dkv::SplitParams& p) {
-  dkv::split_kernel<D, G, BF16, NST><<<grid, dkv::kThreads, smem, s>>>(p);
+  dkv::split_kernel<D, G, BF16, NST, ROPE><<<grid, dkv::kThreads, smem, s>>>(p);
 }
 
-template <int NST>
-SplitVariant pick(int D, int G, bool bf16) {
-#define DKV_NA_CASE(DD, GG)                                                                          \
-  if (D == DD && G == GG)                                                                            \
-    return bf16 ? SplitVariant{&launch_split<DD, GG, true, NST>,                                     \
-                               reinterpret_cast<const void*>(&dkv::split_kernel<DD, GG, true, NST>)} \
-                : SplitVariant{&launch_split<DD, GG, false, NST>,                                    \
-                               reinterpret_cast<const void*>(&dkv::split_kernel<DD, GG, false, NST>)};
+template <int NST, bool ROPE>
+SplitVariant pick_rope(int D, int G, bool bf16) {
+#define DKV_NA_CASE(DD, GG)                                                                                \
+  if (D == DD && G == GG)                                                                                  \
+    return bf16 ? SplitVariant{&launch_split<DD, GG, true, NST, ROPE>,                                     \
+                               reinterpret_cast<const void*>(&dkv::split_kernel<DD, GG, true, NST, ROPE>)} \
+                : SplitVariant{&launch_split<DD, GG, false, NST, ROPE>,                                    \
+                               reinterpret_cast<const void*>(&dkv::split_kernel<DD, GG, false, NST, ROPE>)};
   DKV_NA_CASE(64, 1)
   DKV_NA_CASE(64, 2)
   DKV_NA_CASE(64, 4)
@@ -79,6 +79,11 @@ SplitVariant pick(int D, int G, bool bf16) {
   DKV_NA_CASE(128, 4)
 #undef DKV_NA_CASE
   return {nullptr, nullptr};
+}
+
+template <int NST>
+SplitVariant pick(int D, int G, bool bf16, bool rope) {
+  return rope ? pick_rope<NST, true>(D, G, bf16) : pick_rope<NST, false>(D, G, bf16);
 }
 
 // theta_i(p) = p * base^(-2i/D), written into the scratch array each call.
@@ -170,8 +175,8 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
   } restore{prev, c.device};
 
   const bool bf16 = c.kv_dtype == DKV_KV_BF16;
-  const SplitVariant host_k = pick<kHostStages>(D, G, bf16);
-  const SplitVariant dev_k = pick<kDevStages>(D, G, bf16);
+  const SplitVariant host_k = pick<kHostStages>(D, G, bf16, c.rope_base > 0.0);
+  const SplitVariant dev_k = pick<kDevStages>(D, G, bf16, c.rope_base > 0.0);
   DeviceSetup* st = nullptr;
   int rc = setup_device(c.device, host_k, dev_k, D, &st);
   if (rc != DKV_OK) return rc;
