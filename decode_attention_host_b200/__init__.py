@@ -14,12 +14,15 @@ only bundle those calls for the tests and the benchmark.
 from __future__ import annotations
 
 import ctypes
+import os
 from pathlib import Path
 
 import numpy as np
 
 _PKG = Path(__file__).resolve().parent
-LIB_PATH = _PKG / "libdkv.so"
+# DKV_LIB_PATH selects another build of the same library (e.g. one compiled
+# with different DKV_* build-time knobs) for side-by-side timing.
+LIB_PATH = Path(os.environ.get("DKV_LIB_PATH", str(_PKG / "libdkv.so")))
 
 DKV_OK = 0
 DKV_ERR_INVALID_ARG = -1
@@ -36,7 +39,7 @@ DKV_PLACE_RANDOM = 1
 EXPORTED = ("dkv_create", "dkv_destroy", "dkv_attn_decode", "dkv_get_status", "dkv_last_error_string",
             "dkv_last_launch_count", "dkv_query_plan", "dkv_host_pool_alloc", "dkv_host_pool_free",
             "dkv_plan_blocks", "dkv_pack_kv", "dkv_profile_begin", "dkv_profile_end",
-            "dkv_attn_decode_noalloc")
+            "dkv_attn_decode_noalloc", "dkv_plan_offload")
 
 
 class DkvConfig(ctypes.Structure):
@@ -54,6 +57,11 @@ class DkvPlanParams(ctypes.Structure):
 class DkvPlanResult(ctypes.Structure):
     _fields_ = [("host_split", ctypes.c_int32), ("num_dev_blocks", ctypes.c_int32),
                 ("host_tokens", ctypes.c_int64), ("dev_tokens", ctypes.c_int64)]
+
+
+class DkvOffloadPlan(ctypes.Structure):
+    _fields_ = [("host_fraction", ctypes.c_double), ("step_seconds", ctypes.c_double),
+                ("hbm_bytes_freed", ctypes.c_double), ("time_optimal_fraction", ctypes.c_double)]
 
 
 class DkvError(RuntimeError):
@@ -80,6 +88,7 @@ def _load() -> ctypes.CDLL:
         "dkv_plan_blocks": [c.POINTER(DkvPlanParams), vp, i32, vp, i32, c.POINTER(DkvPlanResult)],
         "dkv_pack_kv": [vp, vp, i64, vp, i32, i32, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp],
         "dkv_profile_begin": [vp, i32],
+        "dkv_plan_offload": [c.c_double, c.c_double, c.c_double, c.c_double, c.POINTER(DkvOffloadPlan)],
         "dkv_attn_decode_noalloc": [c.POINTER(DkvConfig), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32,
                                     i32],
         "dkv_profile_end": [vp, c.POINTER(c.c_float), c.POINTER(i32)],
@@ -168,6 +177,14 @@ def dkv_plan_blocks(params: DkvPlanParams, seq_lens: np.ndarray, block_table: np
     _check(lib.dkv_plan_blocks(ctypes.byref(params), _p(seq_lens), len(seq_lens), _p(block_table),
                                block_table.shape[1], ctypes.byref(res)))
     return res
+
+
+def dkv_plan_offload(kv_bytes: float, host_gbs: float, hbm_gbs: float, hbm_budget_bytes: float = -1.0
+                     ) -> DkvOffloadPlan:
+    plan = DkvOffloadPlan()
+    _check(lib.dkv_plan_offload(float(kv_bytes), float(host_gbs), float(hbm_gbs), float(hbm_budget_bytes),
+                                ctypes.byref(plan)))
+    return plan
 
 
 def dkv_pack_kv(k_logical, v_logical, seq_lens, num_kv_heads, head_dim, block_size, block_table, host_split,

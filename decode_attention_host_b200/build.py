@@ -30,16 +30,21 @@ def up_to_date() -> bool:
     return all(p.stat().st_mtime <= t for p in SOURCES + HEADERS + [Path(__file__)])
 
 
-def build(force: bool = False, verbose: bool = False) -> Path:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, out: Path = LIB, defines: tuple[str, ...] = ()) -> Path:
+    """Compile the library to ``out``; ``defines`` are extra -D build-time knobs (e.g. DKV_DEV_STAGES=2)."""
+    out = Path(out)
+    if not force and not defines and out == LIB and up_to_date():
         return LIB
-    tmp = LIB.with_suffix(f".{os.getpid()}.tmp.so")
-    cmd = [NVCC, *FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", str(tmp), *map(str, SOURCES)]
+    tmp = out.with_suffix(f".{os.getpid()}.tmp.so")
+    cmd = [NVCC, *FLAGS, *(f"-D{d}" for d in defines), *(["-Xptxas", "-v"] if verbose else []), "-o", str(tmp),
+           *map(str, SOURCES)]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    build(force=True, verbose="--verbose" in sys.argv)
-    print(LIB)
+    args = sys.argv[1:]
+    out = Path(args[args.index("--out") + 1]) if "--out" in args else LIB
+    defines = tuple(a[2:] for a in args if a.startswith("-D"))
+    print(build(force=True, verbose="--verbose" in args, out=out, defines=defines))

@@ -52,7 +52,10 @@ struct DeviceGuard {
 };
 
 constexpr int kHostStages = 4;   // ring depth of the zero-copy host kernel (1 CTA per SM, few SMs)
-constexpr int kDevStages = 3;    // ring depth of the HBM kernel (2 CTAs per SM)
+#ifndef DKV_DEV_STAGES
+#define DKV_DEV_STAGES 3
+#endif
+constexpr int kDevStages = DKV_DEV_STAGES;  // ring depth of the HBM kernel (build-time knob)
 constexpr int kDefaultHostCtas = 16;
 constexpr int kMinSplitTokens = 64;
 

@@ -120,6 +120,26 @@ int dkv_plan_blocks(const dkv_plan_params* params, const int32_t* seq_lens, int3
   return DKV_OK;
 }
 
+int dkv_plan_offload(double kv_bytes, double host_gbs, double hbm_gbs, double hbm_budget_bytes,
+                     dkv_offload_plan* plan) {
+  if (!plan || !(kv_bytes > 0.0) || !(host_gbs > 0.0) || !(hbm_gbs > 0.0) || std::isnan(hbm_budget_bytes) ||
+      !std::isfinite(kv_bytes) || !std::isfinite(host_gbs) || !std::isfinite(hbm_gbs))
+    return set_error(DKV_ERR_INVALID_ARG, "dkv_plan_offload: sizes and bandwidths must be positive and finite");
+  const double f_time = host_gbs / (host_gbs + hbm_gbs);
+  double f_cap = 0.0;
+  if (hbm_budget_bytes >= 0.0) f_cap = 1.0 - hbm_budget_bytes / kv_bytes;
+  double f = f_time > f_cap ? f_time : f_cap;
+  if (f > 1.0) f = 1.0;
+  if (f < 0.0) f = 0.0;
+  const double t_host = f * kv_bytes / (host_gbs * 1e9);
+  const double t_dev = (1.0 - f) * kv_bytes / (hbm_gbs * 1e9);
+  plan->host_fraction = f;
+  plan->step_seconds = t_host > t_dev ? t_host : t_dev;
+  plan->hbm_bytes_freed = f * kv_bytes;
+  plan->time_optimal_fraction = f_time;
+  return DKV_OK;
+}
+
 int dkv_pack_kv(const uint16_t* k_logical, const uint16_t* v_logical, int64_t lmax, const int32_t* seq_lens,
                 int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                 const int32_t* block_table, int32_t block_table_stride, int32_t host_split, int32_t num_dev_blocks,

@@ -163,19 +163,23 @@ __device__ __forceinline__ void ldsm_x4_t(const void* p, uint32_t& r0, uint32_t&
                : "r"(smem_u32(p)));
 }
 
-// D(16x8,f32) += A(16x16) * B(16x8), A and B both bf16 or both fp16.
+// D(16x8,f32) += A(16x16) * B(16x8), A and B both bf16 or both fp16, for A
+// whose rows 8..15 are zero: only the C/D rows 0..7 (c[0], c[1]) are kept; the
+// rows 8..15 take a zero input and their outputs are discarded, so they cost
+// no accumulator registers and chain no dependency between calls.
 template <bool BF16>
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma16816_top(float (&c)[2], const uint32_t (&a)[2], uint32_t b0, uint32_t b1) {
+  float d2, d3;
   if constexpr (BF16) {
     asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-                 "{%0,%1,%2,%3};\n"
-                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+                 "{%10,%11,%12,%12};\n"
+                 : "=f"(c[0]), "=f"(c[1]), "=f"(d2), "=f"(d3)
+                 : "r"(a[0]), "r"(0u), "r"(a[1]), "r"(0u), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(0.f));
   } else {
     asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-                 "{%0,%1,%2,%3};\n"
-                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+                 "{%10,%11,%12,%12};\n"
+                 : "=f"(c[0]), "=f"(c[1]), "=f"(d2), "=f"(d3)
+                 : "r"(a[0]), "r"(0u), "r"(a[1]), "r"(0u), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(0.f));
   }
 }
 
@@ -281,6 +285,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   constexpr int TILE = kTileTokens * ROW;      // bytes of one K (or V) tile
   constexpr int CPR = ROW / 16;                // 16-byte chunks per row
   constexpr int NT = D / 8;                    // 8-wide output column tiles of the PV mma
+  static_assert(G <= 4, "hi rows 0..3 and lo rows 4..7 of the PV mma");
   extern __shared__ __align__(128) char smem[];
   __shared__ TileDesc meta[kWarps][NST];
   __shared__ double s_freq[PPL][8];            // [r][li]: base^(-2i/D), i = li*PPL + r
@@ -353,13 +358,22 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   };
 
   // per-unit state.  QX/QY: rotated, pre-scaled queries of this lane's dims.
-  // acc: PV accumulators in mma C layout -- rows 0..G-1 hold the bf16/fp16 "hi"
-  // part of the weights, rows 8..8+G-1 the "lo" remainder; out = row g + row g+8.
+  // acc: PV accumulators in mma C layout (rows 0..7): rows 0..G-1 hold the
+  // bf16/fp16 "hi" part of the weights (lanes 0..4G-1), rows 4..4+G-1 the "lo"
+  // remainder (lanes 16..16+4G-1); out = row g + row 4+g.
   float2 QX[G][NP2], QY[G][NP2];
-  float acc[NT][4];
-  float mrun[G], lrun[G];
+  float acc[NT][2];
+  // After the reduce-scatter of the scores, lane li of every token group owns
+  // head gl of the softmax (G=4: gl = li/2; G=2: li/4; G=1: 0) and keeps that
+  // head's running max and (lane-partial) running sum.
+  constexpr int HL = 8 / G;                    // lanes per head inside a token group
+  const int gl = li / HL;
+  float mrun = -1e30f, lrun = 0.f;
   bool poisoned = false;
   int cur = -1;
+  // RoPE factors carried from one tile to the next when positions continue
+  float2 Cc[NP2], Sc[NP2], NSc[NP2];
+  int next_pos = -1, chain = 0;
 
   auto seeds = [&](int pos, float2 (&C)[NP2], float2 (&S)[NP2]) {
 #pragma unroll
@@ -399,39 +413,52 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
         QX[g][j] = __fmul2_rn(make_float2(xr.x - ys.x, xr.y - ys.y), qs);   // x c - y s
         QY[g][j] = __fmul2_rn(__ffma2_rn(x, S[j], yr), qs);                  // y c + x s
       }
-      mrun[g] = -1e30f;
-      lrun[g] = 0.f;
     }
+    mrun = -1e30f;
+    lrun = 0.f;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = 0.f;
     poisoned = false;
+  };
+
+  // lanes of one head: the HL lanes of a token group (xor < HL) and the 4 groups (xor 8, 16)
+  auto head_sum = [&](float v) {
+#pragma unroll
+    for (int o = 1; o < HL; o <<= 1) v += __shfl_xor_sync(kFull, v, o);
+    v += __shfl_xor_sync(kFull, v, 8);
+    v += __shfl_xor_sync(kFull, v, 16);
+    return v;
+  };
+  auto head_max = [&](float v) {
+#pragma unroll
+    for (int o = 1; o < HL; o <<= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    v = fmaxf(v, __shfl_xor_sync(kFull, v, 8));
+    v = fmaxf(v, __shfl_xor_sync(kFull, v, 16));
+    return v;
   };
 
   auto finalize = [&](int unit, int h) {
     const int bc = unit / p.hkv;
     const int c = bc % p.nsplit;
     const int b = bc / p.nsplit;
-    float ltot[G];
+    const float ltot = head_sum(lrun);
+    // hi rows (lanes 0..15) + lo rows (lanes 16..31) of the same head and columns
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float l = lrun[g];
-      l += __shfl_xor_sync(kFull, l, 8);
-      l += __shfl_xor_sync(kFull, l, 16);
-      ltot[g] = l;
+    for (int n = 0; n < NT; ++n) {
+      acc[n][0] += __shfl_xor_sync(kFull, acc[n][0], 16);
+      acc[n][1] += __shfl_xor_sync(kFull, acc[n][1], 16);
     }
+    // the output lanes of head gT take its sum and max from lane gT * HL
+    const float l = __shfl_sync(kFull, ltot, (gT & 3) * HL);
+    const float M = __shfl_sync(kFull, mrun, (gT & 3) * HL);
     if (gT < G) {
-      float l = ltot[0], M = mrun[0];
-#pragma unroll
-      for (int g = 1; g < G; ++g)
-        if (gT == g) { l = ltot[g]; M = mrun[g]; }
       const size_t row = (static_cast<size_t>(b) * p.hq + h * G + gT) * p.nslots + p.slot_base + c;
       float* o = p.part_o + row * D;
       const float qnan = __int_as_float(0x7fc00000);
       const float inv = poisoned ? qnan : (l > 0.f ? 1.f / l : 0.f);
 #pragma unroll
       for (int n = 0; n < NT; ++n)
-        *reinterpret_cast<float2*>(o + 8 * n + 2 * cT) =
-            make_float2((acc[n][0] + acc[n][2]) * inv, (acc[n][1] + acc[n][3]) * inv);
+        *reinterpret_cast<float2*>(o + 8 * n + 2 * cT) = make_float2(acc[n][0] * inv, acc[n][1] * inv);
       if (cT == 0) p.part_lse[row] = poisoned ? qnan : (l > 0.f ? M + __log2f(l) : -INFINITY);
     }
   };
@@ -443,11 +470,22 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     // ---- scores: rotate K rows on the fly (CUDA cores, fp32 pairs)
     float2 C[NP2], S[NP2], NS[NP2];
     if constexpr (ROPE) {
-      seeds(d.p0 + tg, C, S);
+      if (d.p0 == next_pos && chain < 4) {
 #pragma unroll
-      for (int j = 0; j < NP2; ++j) NS[j] = make_float2(-S[j].x, -S[j].y);
+        for (int j = 0; j < NP2; ++j) {
+          C[j] = Cc[j];
+          S[j] = Sc[j];
+          NS[j] = NSc[j];
+        }
+        ++chain;
+      } else {
+        seeds(d.p0 + tg, C, S);
+#pragma unroll
+        for (int j = 0; j < NP2; ++j) NS[j] = make_float2(-S[j].x, -S[j].y);
+        chain = 1;
+      }
     }
-    float sc[4][G];
+    float v[4 * G];  // partial scores, index g * 4 + m
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int t = tg + 4 * m;
@@ -461,77 +499,115 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
           const float2 x = X[j], y = Y[j];
           X[j] = __ffma2_rn(y, NS[j], __fmul2_rn(x, C[j]));   // x c - y s
           Y[j] = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));    // y c + x s
-          if (m < 3) {  // advance 4 positions: (C + iS)(E + iF)
-            const float2 e = s_e[j][li], f = s_f[j][li], nf = s_nf[j][li];
-            const float2 cn = __ffma2_rn(NS[j], f, __fmul2_rn(C[j], e));
-            const float2 sn = __ffma2_rn(C[j], f, __fmul2_rn(S[j], e));
-            NS[j] = __ffma2_rn(C[j], nf, __fmul2_rn(NS[j], e));
-            C[j] = cn;
-            S[j] = sn;
-          }
+          // advance 4 positions: (C + iS)(E + iF); after m = 3 this is the
+          // first token of the tile 16 positions on
+          const float2 e = s_e[j][li], f = s_f[j][li], nf = s_nf[j][li];
+          const float2 cn = __ffma2_rn(NS[j], f, __fmul2_rn(C[j], e));
+          const float2 sn = __ffma2_rn(C[j], f, __fmul2_rn(S[j], e));
+          NS[j] = __ffma2_rn(C[j], nf, __fmul2_rn(NS[j], e));
+          C[j] = cn;
+          S[j] = sn;
         }
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float2 a = __fmul2_rn(QX[g][0], X[0]);
-        a = __ffma2_rn(QY[g][0], Y[0], a);
+        float2 ax = __fmul2_rn(QX[g][0], X[0]);
+        float2 ay = __fmul2_rn(QY[g][0], Y[0]);
 #pragma unroll
         for (int j = 1; j < NP2; ++j) {
-          a = __ffma2_rn(QX[g][j], X[j], a);
-          a = __ffma2_rn(QY[g][j], Y[j], a);
+          ax = __ffma2_rn(QX[g][j], X[j], ax);
+          ay = __ffma2_rn(QY[g][j], Y[j], ay);
         }
-        sc[m][g] = a.x + a.y;
+        const float2 a = __fadd2_rn(ax, ay);
+        v[g * 4 + m] = a.x + a.y;
       }
     }
+    if constexpr (ROPE) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float a = sc[m][g];
-        a += __shfl_xor_sync(kFull, a, 1);
-        a += __shfl_xor_sync(kFull, a, 2);
-        a += __shfl_xor_sync(kFull, a, 4);
-        sc[m][g] = (tg + 4 * m) < nvalid ? a : -INFINITY;
+      for (int j = 0; j < NP2; ++j) {
+        Cc[j] = C[j];
+        Sc[j] = S[j];
+        NSc[j] = NS[j];
       }
-    // ---- online softmax, one running max per head for the whole warp
-    float alpha[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float tm = fmaxf(fmaxf(sc[0][g], sc[1][g]), fmaxf(sc[2][g], sc[3][g]));
-      tm = fmaxf(tm, __shfl_xor_sync(kFull, tm, 8));
-      tm = fmaxf(tm, __shfl_xor_sync(kFull, tm, 16));
-      const float mx = fmaxf(mrun[g], tm);
-      alpha[g] = ex2(mrun[g] - mx);
-      float pv[4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) pv[m] = ex2(sc[m][g] - mx);
-      if (li == 0) *reinterpret_cast<float4*>(&s_p[warp][g][tg][0]) = make_float4(pv[0], pv[1], pv[2], pv[3]);
-      lrun[g] = lrun[g] * alpha[g] + ((pv[0] + pv[1]) + (pv[2] + pv[3]));
-      mrun[g] = mx;
+      next_pos = d.p0 + kTileTokens;
     }
+    // ---- reduce-scatter over the 8 lanes of the token group: halve the value
+    // set at each xor step; lane li ends with scores g*4+m = li*(4G/8) + k
+    constexpr int NV = 4 * G;
+    constexpr int NH = NV >= 8 ? NV / 8 : 1;  // values held per lane at the end
+#pragma unroll
+    for (int b = 4, n = NV; b >= 1; b >>= 1) {
+      if (n > 1) {
+        const bool up = (li & b) != 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (i < n / 2) {
+            const float send = up ? v[i] : v[i + n / 2];
+            const float keep = up ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(kFull, send, b);
+          }
+        }
+        n >>= 1;
+      } else {
+        v[0] += __shfl_xor_sync(kFull, v[0], b);
+      }
+    }
+    // this lane's tokens (G=4: m = 2(li&1)+k; G=2: m = li&3; G=1: m = li>>1)
+    float sc[NH];
+    int mt[NH];
+#pragma unroll
+    for (int k = 0; k < NH; ++k) {
+      const int j = (G == 4) ? (li * 2 + k) : (G == 2 ? li : (li >> 1));
+      mt[k] = j & 3;
+      sc[k] = (tg + 4 * mt[k]) < nvalid ? v[k] : -INFINITY;
+    }
+    // ---- online softmax for head gl (max shared by the head's lanes)
+    float tm = sc[0];
+#pragma unroll
+    for (int k = 1; k < NH; ++k) tm = fmaxf(tm, sc[k]);
+    tm = head_max(tm);
+    const float mx = fmaxf(mrun, tm);
+    const float alpha = ex2(mrun - mx);
+    float psum = 0.f;
+    float pv[NH];
+#pragma unroll
+    for (int k = 0; k < NH; ++k) {
+      pv[k] = ex2(sc[k] - mx);
+      psum += pv[k];
+    }
+    if constexpr (G == 4) {
+      *reinterpret_cast<float2*>(&s_p[warp][gl][tg][mt[0]]) = make_float2(pv[0], pv[1]);
+    } else if constexpr (G == 2) {
+      s_p[warp][gl][tg][mt[0]] = pv[0];
+    } else {
+      if ((li & 1) == 0) s_p[warp][0][tg][mt[0]] = pv[0];
+      if (li & 1) psum = 0.f;  // the odd lane holds a duplicate of its even neighbour's token
+    }
+    lrun = lrun * alpha + psum;
+    mrun = mx;
     __syncwarp();
-    // ---- PV on the tensor cores: A = weights (hi rows 0..G-1, lo rows 8..), B = V
-    uint32_t a[4] = {0u, 0u, 0u, 0u};
-    float al = 1.f;
-    if (gT < G) {
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-        if (gT == g) al = alpha[g];
-      // tokens 2c, 2c+1 (a) and 2c+8, 2c+9 (b); token t lives at [t % 4][t / 4]
-      const float* sp = &s_p[warp][gT][0][0];
+    // ---- PV on the tensor cores.  A rows 0..7 (lane >> 2): rows 0..3 hi,
+    // rows 4..7 lo, of head (lane >> 2) & 3; B = V from the swizzled tile.
+    uint32_t a[2] = {0u, 0u};
+    const int gA = gT & 3;
+    const float al = __shfl_sync(kFull, alpha, gA * HL);
+    if (gA < G) {
+      // tokens 2c, 2c+1 (a[0]) and 2c+8, 2c+9 (a[1]); token t lives at [t % 4][t / 4]
+      const float* sp = &s_p[warp][gA][0][0];
       const int t0 = 2 * cT;
       const float2 pa = make_float2(sp[(t0 & 3) * 4 + (t0 >> 2)], sp[((t0 + 1) & 3) * 4 + (t0 >> 2)]);
       const float2 pb = make_float2(sp[(t0 & 3) * 4 + (t0 >> 2) + 2], sp[((t0 + 1) & 3) * 4 + (t0 >> 2) + 2]);
-      split_hi_lo<BF16>(pa, a[0], a[1]);
-      split_hi_lo<BF16>(pb, a[2], a[3]);
+      uint32_t ha, la, hb, lb;
+      split_hi_lo<BF16>(pa, ha, la);
+      split_hi_lo<BF16>(pb, hb, lb);
+      a[0] = lane < 16 ? ha : la;
+      a[1] = lane < 16 ? hb : lb;
     }
     if (al != 1.f) {
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         acc[n][0] *= al;
         acc[n][1] *= al;
-        acc[n][2] *= al;
-        acc[n][3] *= al;
       }
     }
     const int vrow = (lane & 7) | (lane & 8);
@@ -539,8 +615,8 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     for (int qd = 0; qd < D / 16; ++qd) {
       uint32_t b0, b1, b2, b3;
       ldsm_x4_t(sv + swz<ROW>(vrow, 2 * qd + (lane >> 4)), b0, b1, b2, b3);
-      mma16816<BF16>(acc[2 * qd], a, b0, b1);
-      mma16816<BF16>(acc[2 * qd + 1], a, b2, b3);
+      mma16816_top<BF16>(acc[2 * qd], a, b0, b1);
+      mma16816_top<BF16>(acc[2 * qd + 1], a, b2, b3);
     }
   };
 

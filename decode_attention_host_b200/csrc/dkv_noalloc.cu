@@ -33,7 +33,10 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[DKV_NOALLOC_SCR
 
 constexpr int kMaxDevices = 64;
 constexpr int kHostStages = 4;
-constexpr int kDevStages = 3;
+#ifndef DKV_DEV_STAGES
+#define DKV_DEV_STAGES 3
+#endif
+constexpr int kDevStages = DKV_DEV_STAGES;
 constexpr int kHostCtas = 16;
 constexpr int kMinSplitTokens = 64;
 constexpr size_t kStatusOffset = 0;     // int32 status word

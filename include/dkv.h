@@ -236,6 +236,33 @@ DKV_API int dkv_plan_blocks(const dkv_plan_params* params, const int32_t* seq_le
                     int32_t block_table_stride, dkv_plan_result* result);
 
 /*
+ * dkv_plan_offload -- choose the host fraction of the KV cache (SplitKernel
+ * README, Key Features: placement / offloading-ratio utilities; DirectKV
+ * README, Figure mapping, Fig 11b: GPU memory freed at long context).
+ * With X = total KV bytes, the modelled step time of a placement with host
+ * fraction f is T(f) = max(f*X / host_gbs, (1-f)*X / hbm_gbs): the zero-copy
+ * host stream and the HBM kernel run concurrently and the slower one sets the
+ * step.  T falls while the HBM side dominates and rises once PCIe does, so the
+ * time-optimal fraction is f* = host_gbs / (host_gbs + hbm_gbs).  An HBM budget
+ * for the cache forces f >= 1 - budget/X.  The plan is f = max(f*, that bound),
+ * capped at 1.
+ *   kv_bytes        X > 0
+ *   host_gbs        measured host read bandwidth the kernel achieves (> 0)
+ *   hbm_gbs         measured HBM read bandwidth (> 0)
+ *   hbm_budget_bytes  HBM bytes the cache may occupy; < 0 means unlimited
+ * Out: host_fraction, predicted step seconds, HBM bytes freed (f*X) and the
+ * time-optimal fraction f*.  Pure host arithmetic; errors: INVALID_ARG. */
+typedef struct dkv_offload_plan {
+  double host_fraction;
+  double step_seconds;
+  double hbm_bytes_freed;
+  double time_optimal_fraction;
+} dkv_offload_plan;
+
+DKV_API int dkv_plan_offload(double kv_bytes, double host_gbs, double hbm_gbs, double hbm_budget_bytes,
+                             dkv_offload_plan* plan);
+
+/*
  * dkv_pack_kv -- write logical K/V into the paged pools following a table.
  *   k_logical, v_logical  host, 16-bit [batch][Hkv][lmax][D]
  *   seq_lens, block_table host, as in dkv_plan_blocks

@@ -38,7 +38,8 @@ def test_struct_layout_matches_header(tmp_path):
     src = tmp_path / "layout.c"
     fields = {"dkv_config": [f for f, _ in dkv.DkvConfig._fields_],
               "dkv_plan_params": [f for f, _ in dkv.DkvPlanParams._fields_],
-              "dkv_plan_result": [f for f, _ in dkv.DkvPlanResult._fields_]}
+              "dkv_plan_result": [f for f, _ in dkv.DkvPlanResult._fields_],
+              "dkv_offload_plan": [f for f, _ in dkv.DkvOffloadPlan._fields_]}
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "dkv.h"', "int main(void) {"]
     for st, fs in fields.items():
         lines.append(f'printf("{st} size %zu\\n", sizeof({st}));')
@@ -53,7 +54,7 @@ def test_struct_layout_matches_header(tmp_path):
         *key, val = line.split()
         got[tuple(key)] = int(val)
     for st, cls in (("dkv_config", dkv.DkvConfig), ("dkv_plan_params", dkv.DkvPlanParams),
-                    ("dkv_plan_result", dkv.DkvPlanResult)):
+                    ("dkv_plan_result", dkv.DkvPlanResult), ("dkv_offload_plan", dkv.DkvOffloadPlan)):
         assert got[(st, "size")] == ctypes.sizeof(cls)
         for f, _ in cls._fields_:
             assert got[(st, f)] == getattr(cls, f).offset, (st, f)

@@ -124,3 +124,41 @@ def test_pack_places_every_token_where_the_table_says(S, f, shuffle):
             assert np.array_equal(tile_k[:, :n], k[b, :, j * S:j * S + n])
             assert np.array_equal(tile_v[:, :n], v[b, :, j * S:j * S + n])
             assert not tile_k[:, n:].any() and not tile_v[:, n:].any()
+
+
+# ----------------------------------------------------------------------------- offload-ratio planner
+
+def test_offload_time_optimal_fraction_balances_the_two_sides():
+    plan = dkv.dkv_plan_offload(1 << 30, 51.5, 6547.8)
+    f = 51.5 / (51.5 + 6547.8)
+    assert abs(plan.time_optimal_fraction - f) < 1e-15 and abs(plan.host_fraction - f) < 1e-15
+    t_host = f * (1 << 30) / 51.5e9
+    t_dev = (1 - f) * (1 << 30) / 6547.8e9
+    assert abs(t_host - t_dev) < 1e-15 and abs(plan.step_seconds - t_host) < 1e-15
+    assert abs(plan.hbm_bytes_freed - f * (1 << 30)) < 1e-3
+
+
+def test_offload_budget_forces_more_onto_the_host():
+    X = 4 * (1 << 30)
+    plan = dkv.dkv_plan_offload(X, 51.5, 6547.8, hbm_budget_bytes=0.1 * X)   # long-context case: 10% fits
+    assert abs(plan.host_fraction - 0.9) < 1e-12
+    assert abs(plan.hbm_bytes_freed - 0.9 * X) < 1e-3
+    assert abs(plan.step_seconds - 0.9 * X / 51.5e9) < 1e-12
+    # a budget larger than the cache leaves the time-optimal split; a zero budget puts everything on the host
+    assert abs(dkv.dkv_plan_offload(X, 51.5, 6547.8, 2 * X).host_fraction - plan.time_optimal_fraction) < 1e-15
+    assert dkv.dkv_plan_offload(X, 51.5, 6547.8, 0.0).host_fraction == 1.0
+
+
+def test_offload_step_time_is_minimal_at_the_plan():
+    X, hb, db = 1e9, 50.0, 7000.0
+    plan = dkv.dkv_plan_offload(X, hb, db)
+    for f in np.linspace(0, 1, 101):
+        t = max(f * X / (hb * 1e9), (1 - f) * X / (db * 1e9))
+        assert t >= plan.step_seconds - 1e-15
+
+
+@pytest.mark.parametrize("args", [(0, 50, 7000, -1), (1e9, 0, 7000, -1), (1e9, 50, -1, -1), (float("inf"), 50, 7000, -1),
+                                  (1e9, 50, 7000, float("nan"))])
+def test_offload_rejects_bad_inputs(args):
+    with pytest.raises(dkv.DkvError):
+        dkv.dkv_plan_offload(*args)
