@@ -260,7 +260,7 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   const bool rope = c.rope_base > 0.0;
   h->host_kernel = pick_split<kHostStages>(c.head_dim, G, bf16, rope);
   h->dev_kernel = pick_split<kDevStages>(c.head_dim, G, bf16, rope);
-  h->merge = c.head_dim == 64 ? &launch_merge<64, 4> : &launch_merge<128, 2>;
+  h->merge = c.head_dim == 64 ? &launch_merge<64, 16> : &launch_merge<128, 8>;
 
   auto bail = [&](int code) {
     release(h);
@@ -268,7 +268,7 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   };
   cudaError_t e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, c.device);
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaDeviceGetAttribute"));
-  h->units_target = h->sm_count * 16;
+  h->units_target = h->sm_count * 8;  // one unit per warp of a full wave (2 CTAs x 4 warps per SM)
   h->part_rows = 2ull * G * (static_cast<size_t>(h->units_target) + static_cast<size_t>(c.max_batch) * c.num_kv_heads);
   e = cudaFuncSetAttribute(h->host_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(split_smem(c.head_dim, kHostStages)));
@@ -419,7 +419,8 @@ int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const voi
     dp.id_hi = host_split + num_dev_blocks;
     dp.slot_base = nsplit;
     if ((rc = prof_mark(h, 1, s, false)) != DKV_OK) return rc;
-    h->dev_kernel.fn(dim3(unit_ctas), split_smem(c.head_dim, kDevStages), s, dp);
+    const int dev_ctas = unit_ctas < 2 * h->sm_count ? unit_ctas : 2 * h->sm_count;  // one resident wave
+    h->dev_kernel.fn(dim3(dev_ctas), split_smem(c.head_dim, kDevStages), s, dp);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 1, s, true)) != DKV_OK) return rc;
     ++launches;

@@ -712,7 +712,7 @@ __global__ void __launch_bounds__(NG * D) merge_kernel(const MergeParams p) {
   const int d = tid % D;
   const int grp = tid / D;
   float acc = 0.f;
-#pragma unroll 4
+#pragma unroll 2
   for (int i = grp; i < p.nslots; i += NG) {
     const float wi = wts[i];
     if (wi != 0.f) acc = fmaf(wi, o[static_cast<size_t>(i) * D + d], acc);

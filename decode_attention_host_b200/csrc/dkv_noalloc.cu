@@ -206,7 +206,7 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
   // split plan: as in dkv_attn_decode, then narrowed until the partials fit the scratch
   const int nblk = block_table_stride < c.max_blocks_per_seq ? block_table_stride : c.max_blocks_per_seq;
   const long per = static_cast<long>(batch) * c.num_kv_heads;
-  const long units_target = static_cast<long>(st->sm_count) * 16;
+  const long units_target = static_cast<long>(st->sm_count) * 8;
   int target = static_cast<int>((units_target + per - 1) / per);
   if (target < 1) target = 1;
   int bps = (nblk + target - 1) / target;
@@ -273,7 +273,8 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
     dp.id_lo = host_split;
     dp.id_hi = host_split + num_dev_blocks;
     dp.slot_base = nsplit;
-    dev_k.launch(dim3(unit_ctas), split_smem(D, kDevStages), s, dp);
+    const int dev_ctas = unit_ctas < 2 * st->sm_count ? unit_ctas : 2 * st->sm_count;  // one resident wave
+    dev_k.launch(dim3(dev_ctas), split_smem(D, kDevStages), s, dp);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_error(e, "HBM kernel launch");
   }
   dkv::MergeParams mp{};
@@ -285,9 +286,9 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
   mp.has_host = host_split > 0;
   mp.has_dev = num_dev_blocks > 0;
   if (D == 64)
-    dkv::merge_kernel<64, 4><<<batch * c.num_q_heads, 4 * 64, nslots * sizeof(float), s>>>(mp);
+    dkv::merge_kernel<64, 16><<<batch * c.num_q_heads, 16 * 64, nslots * sizeof(float), s>>>(mp);
   else
-    dkv::merge_kernel<128, 2><<<batch * c.num_q_heads, 2 * 128, nslots * sizeof(float), s>>>(mp);
+    dkv::merge_kernel<128, 8><<<batch * c.num_q_heads, 8 * 128, nslots * sizeof(float), s>>>(mp);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_error(e, "merge kernel launch");
   if (status_out &&
       (e = cudaMemcpyAsync(status_out, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
