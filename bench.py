@@ -45,6 +45,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama3_8b")
     ap.add_argument("--impl", choices=("dkv", "reference"), default="dkv")
+    ap.add_argument("--mode", choices=("zero_copy", "staged"), default="zero_copy",
+                    help="staged: the prefetch comparator (host pool copied into HBM each step)")
     ap.add_argument("--host-ctas", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -273,8 +275,19 @@ def run_dkv(args):
     stream = torch.cuda.current_stream(device)
     b_pcie = measure_pcie_gbs(device)
 
+    if args.mode == "staged":
+        blk = w.num_kv_heads * w.block_size * w.head_dim
+        k_stage = torch.empty(max(1, kv.host_split * blk), dtype=torch.int16, device=device)
+        v_stage = torch.empty_like(k_stage)
+
+        def step():
+            attn.staged(q_dev, kv, out, k_stage, v_stage, stream)
+    else:
+        def step():
+            attn(q_dev, kv, out, stream)
+
     for _ in range(args.warmup):
-        attn(q_dev, kv, out, stream)
+        step()
     torch.cuda.synchronize(device)
     if attn.status() != 0:
         raise RuntimeError("device status nonzero after warm-up")
@@ -288,7 +301,7 @@ def run_dkv(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        attn(q_dev, kv, out, stream)
+        step()
     e1.record(stream)
     torch.cuda.synchronize(device)
     kernel_ms, kernel_counts = dkv.dkv_profile_end(attn.handle)
@@ -312,7 +325,7 @@ def run_dkv(args):
             q_dev.copy_(q_h, non_blocking=True)
             kv.seq_lens_dev.copy_(lens_h, non_blocking=True)
             kv.table_dev.copy_(table_h, non_blocking=True)
-            attn(q_dev, kv, out, stream)
+            step()
             out_h.copy_(out, non_blocking=True)
 
         for _ in range(args.warmup):
@@ -355,8 +368,9 @@ def run_dkv(args):
     hbm_src = "MEASURED_PEAKS.json hbm_gbs (copy, measured)" if "hbm_gbs" in peaks else "fallback 6650 GB/s"
 
     kernels = []
+    host_name = "staged_copy_then_hbm" if args.mode == "staged" else "host_stream"
     for idx, name, nbytes, bound, peak, unit_src in (
-            (0, "host_stream", host_bytes, "pcie", b_pcie, "pinned H2D cudaMemcpyAsync measured in this run"),
+            (0, host_name, host_bytes, "pcie", b_pcie, "pinned H2D cudaMemcpyAsync measured in this run"),
             (1, "hbm_split_k", dev_bytes, "hbm", hbm_peak, hbm_src)):
         if kernel_counts[idx] == 0:
             continue
@@ -386,7 +400,7 @@ def run_dkv(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
-        "config": dict(workload_config(w, world), host_bytes=host_bytes, dev_bytes=dev_bytes,
+        "config": dict(workload_config(w, world), host_bytes=host_bytes, dev_bytes=dev_bytes, mode=args.mode,
                        l2="inputs larger than L2: %.0f MiB of KV per step vs 126 MB L2" % ((host_bytes + dev_bytes) / 2**20)),
         "roofline": ({k2: dominant[k2] for k2 in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
                      if dominant else None),

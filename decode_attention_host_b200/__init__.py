@@ -39,7 +39,7 @@ DKV_PLACE_RANDOM = 1
 EXPORTED = ("dkv_create", "dkv_destroy", "dkv_attn_decode", "dkv_get_status", "dkv_last_error_string",
             "dkv_last_launch_count", "dkv_query_plan", "dkv_host_pool_alloc", "dkv_host_pool_free",
             "dkv_plan_blocks", "dkv_pack_kv", "dkv_profile_begin", "dkv_profile_end",
-            "dkv_attn_decode_noalloc", "dkv_plan_offload")
+            "dkv_attn_decode_noalloc", "dkv_plan_offload", "dkv_attn_decode_staged")
 
 
 class DkvConfig(ctypes.Structure):
@@ -79,6 +79,7 @@ def _load() -> ctypes.CDLL:
         "dkv_create": [c.POINTER(DkvConfig), c.POINTER(vp)],
         "dkv_destroy": [vp],
         "dkv_attn_decode": [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32],
+        "dkv_attn_decode_staged": [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, vp, vp],
         "dkv_get_status": [vp, c.POINTER(i32)],
         "dkv_last_error_string": [],
         "dkv_last_launch_count": [vp, c.POINTER(i32)],
@@ -136,6 +137,13 @@ def dkv_attn_decode(h, q, k_host, v_host, k_dev, v_dev, block_table, seq_lens, h
     _check(lib.dkv_attn_decode(h, _p(q), _p(k_host), _p(v_host), _p(k_dev), _p(v_dev), _p(block_table),
                                _p(seq_lens), int(host_split), _p(out), stream, int(batch),
                                int(block_table_stride), int(num_dev_blocks)))
+
+
+def dkv_attn_decode_staged(h, q, k_host, v_host, k_dev, v_dev, block_table, seq_lens, host_split, out, stream,
+                           batch, block_table_stride, num_dev_blocks, k_stage, v_stage) -> None:
+    _check(lib.dkv_attn_decode_staged(h, _p(q), _p(k_host), _p(v_host), _p(k_dev), _p(v_dev), _p(block_table),
+                                      _p(seq_lens), int(host_split), _p(out), stream, int(batch),
+                                      int(block_table_stride), int(num_dev_blocks), _p(k_stage), _p(v_stage)))
 
 
 def dkv_get_status(h: int) -> int:
@@ -307,6 +315,16 @@ class DecodeAttention:
                         kv.k_dev if kv.num_dev_blocks else None, kv.v_dev if kv.num_dev_blocks else None,
                         kv.table_dev, kv.seq_lens_dev, kv.host_split, out, stream.cuda_stream, kv.batch,
                         kv.stride, kv.num_dev_blocks)
+
+    def staged(self, q, kv: PagedKV, out, k_stage, v_stage, stream=None) -> None:
+        """The staged-prefetch comparator: copy the host pools into HBM, then run HBM kernels only."""
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(q.device)
+        dkv_attn_decode_staged(self.handle, q, kv.k_host.ptr or None, kv.v_host.ptr or None,
+                               kv.k_dev if kv.num_dev_blocks else None, kv.v_dev if kv.num_dev_blocks else None,
+                               kv.table_dev, kv.seq_lens_dev, kv.host_split, out, stream.cuda_stream, kv.batch,
+                               kv.stride, kv.num_dev_blocks, k_stage, v_stage)
 
     def status(self) -> int:
         return dkv_get_status(self.handle)

@@ -126,7 +126,7 @@ struct dkv_handle {
   SplitEntry host_kernel{}, dev_kernel{};
   MergeFn merge = nullptr;
   const void* ok_host[2] = {nullptr, nullptr};
-  const void* ok_dev[2] = {nullptr, nullptr};
+  const void* ok_dev[4] = {nullptr, nullptr, nullptr, nullptr};
   int last_launches = 0;
   // per-kernel event pairs while profiling: [kernel][call] -> (start, stop)
   int prof_capacity = 0;
@@ -327,10 +327,18 @@ int dkv_last_launch_count(const dkv_handle* h, int32_t* count) {
   return DKV_OK;
 }
 
-int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const void* v_host, const void* k_dev,
-                    const void* v_dev, const int32_t* block_table, const int32_t* seq_lens, int32_t host_split,
-                    float* out, dkv_stream_t stream, int32_t batch, int32_t block_table_stride,
-                    int32_t num_dev_blocks) {
+}  // extern "C"
+
+namespace {
+
+// One decode step.  k_stage == nullptr: zero-copy (host kernel on the aux
+// stream reads the mapped host pools).  Otherwise the staged-prefetch
+// comparator: the host pools are first copied into k_stage / v_stage.
+int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v_host, const void* k_dev,
+                const void* v_dev, const int32_t* block_table, const int32_t* seq_lens, int32_t host_split, float* out,
+                dkv_stream_t stream, int32_t batch, int32_t block_table_stride, int32_t num_dev_blocks, void* k_stage,
+                void* v_stage) {
+  const bool staged = k_stage != nullptr || v_stage != nullptr;
   if (!h) return fail(DKV_ERR_INVALID_ARG, "dkv_attn_decode: null handle");
   if (batch < 0 || batch > h->cfg.max_batch) return fail(DKV_ERR_INVALID_ARG, "batch outside [0, max_batch]");
   if (batch == 0) {
@@ -359,6 +367,13 @@ int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const voi
   if (num_dev_blocks > 0) {
     if ((rc = check_dev_pool(h, k_dev, 0)) != DKV_OK) return rc;
     if ((rc = check_dev_pool(h, v_dev, 1)) != DKV_OK) return rc;
+  }
+  if (staged && host_split > 0) {
+    if (!k_stage || !v_stage) return fail(DKV_ERR_INVALID_ARG, "staging pools must both be given");
+    if ((reinterpret_cast<uintptr_t>(k_stage) | reinterpret_cast<uintptr_t>(v_stage)) % 16 != 0)
+      return fail(DKV_ERR_INVALID_ARG, "staging pools must be 16-byte aligned");
+    if ((rc = check_dev_pool(h, k_stage, 2)) != DKV_OK) return rc;
+    if ((rc = check_dev_pool(h, v_stage, 3)) != DKV_OK) return rc;
   }
 
   const dkv_config& c = h->cfg;
@@ -394,7 +409,24 @@ int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const voi
   const int unit_ctas = (n_units + dkv::kWarps - 1) / dkv::kWarps;
   int launches = 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (host_split > 0) {
+  if (host_split > 0 && staged) {
+    // copy engine: pinned host pools -> HBM staging pools, then the HBM kernel reads them
+    const size_t bytes = static_cast<size_t>(host_split) * c.num_kv_heads * c.block_size * c.head_dim * 2;
+    if ((rc = prof_mark(h, 0, s, false)) != DKV_OK) return rc;
+    DKV_CUDA(cudaMemcpyAsync(k_stage, k_host, bytes, cudaMemcpyHostToDevice, s));
+    DKV_CUDA(cudaMemcpyAsync(v_stage, v_host, bytes, cudaMemcpyHostToDevice, s));
+    dkv::SplitParams hp = sp;
+    hp.k_pool = static_cast<const uint16_t*>(k_stage);
+    hp.v_pool = static_cast<const uint16_t*>(v_stage);
+    hp.id_lo = 0;
+    hp.id_hi = host_split;
+    hp.slot_base = 0;
+    const int dev_ctas = unit_ctas < 2 * h->sm_count ? unit_ctas : 2 * h->sm_count;
+    h->dev_kernel.fn(dim3(dev_ctas), split_smem(c.head_dim, kDevStages), s, hp);
+    DKV_CUDA(cudaGetLastError());
+    if ((rc = prof_mark(h, 0, s, true)) != DKV_OK) return rc;
+    ++launches;
+  } else if (host_split > 0) {
     DKV_CUDA(cudaEventRecord(h->ev_fork, s));
     DKV_CUDA(cudaStreamWaitEvent(h->aux, h->ev_fork, 0));
     dkv::SplitParams hp = sp;
@@ -425,7 +457,7 @@ int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const voi
     if ((rc = prof_mark(h, 1, s, true)) != DKV_OK) return rc;
     ++launches;
   }
-  if (host_split > 0) DKV_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
+  if (host_split > 0 && !staged) DKV_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
   dkv::MergeParams mp{};
   mp.part_o = h->part_o;
   mp.part_lse = h->part_lse;
@@ -441,6 +473,29 @@ int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const voi
   ++launches;
   h->last_launches = launches;
   return DKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const void* v_host, const void* k_dev,
+                    const void* v_dev, const int32_t* block_table, const int32_t* seq_lens, int32_t host_split,
+                    float* out, dkv_stream_t stream, int32_t batch, int32_t block_table_stride,
+                    int32_t num_dev_blocks) {
+  return decode_impl(h, q, k_host, v_host, k_dev, v_dev, block_table, seq_lens, host_split, out, stream, batch,
+                     block_table_stride, num_dev_blocks, nullptr, nullptr);
+}
+
+int dkv_attn_decode_staged(dkv_handle* h, const float* q, const void* k_host, const void* v_host, const void* k_dev,
+                           const void* v_dev, const int32_t* block_table, const int32_t* seq_lens,
+                           int32_t host_split, float* out, dkv_stream_t stream, int32_t batch,
+                           int32_t block_table_stride, int32_t num_dev_blocks, void* k_stage, void* v_stage) {
+  if (host_split > 0 && (!k_stage || !v_stage))
+    return fail(DKV_ERR_INVALID_ARG, "dkv_attn_decode_staged: staging pools are null");
+  return decode_impl(h, q, k_host, v_host, k_dev, v_dev, block_table, seq_lens, host_split, out, stream, batch,
+                     block_table_stride, num_dev_blocks, host_split > 0 ? k_stage : nullptr,
+                     host_split > 0 ? v_stage : nullptr);
 }
 
 int dkv_profile_begin(dkv_handle* h, int32_t max_calls) {

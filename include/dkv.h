@@ -122,6 +122,25 @@ DKV_API int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, c
                     const int32_t* seq_lens, int32_t host_split, float* out, dkv_stream_t stream,
                     int32_t batch, int32_t block_table_stride, int32_t num_dev_blocks);
 
+/*
+ * dkv_attn_decode_staged -- the staged-prefetch comparator: the design the
+ * zero-copy method is measured against (SplitKernel README, Overview:
+ * prefetch-based offloading that first moves offloaded data back into HBM;
+ * DirectKV README, Artifact Evaluation: the Pie / FlexGen prefetch baselines).
+ * The first host_split blocks of the host pools are copied into the device
+ * staging pools k_stage / v_stage with cudaMemcpyAsync (copy engine, pinned
+ * host -> HBM) on `stream`, then both pools are read by the HBM split-K
+ * kernel and merged.  Same arguments and results as dkv_attn_decode, plus:
+ *   k_stage, v_stage  device memory (HBM) of >= host_split blocks each, pool
+ *                     layout, 16-byte aligned; owned by the caller.
+ * It costs host_split blocks of HBM and one HBM write + read of them per call;
+ * dkv_attn_decode needs neither.  Errors: as dkv_attn_decode. */
+DKV_API int dkv_attn_decode_staged(dkv_handle* h, const float* q, const void* k_host, const void* v_host,
+                                   const void* k_dev, const void* v_dev, const int32_t* block_table,
+                                   const int32_t* seq_lens, int32_t host_split, float* out, dkv_stream_t stream,
+                                   int32_t batch, int32_t block_table_stride, int32_t num_dev_blocks, void* k_stage,
+                                   void* v_stage);
+
 /* dkv_get_status -- synchronise the handle's device, return the accumulated
  * DKV_STATUS_* bits in *status and clear them. */
 DKV_API int dkv_get_status(dkv_handle* h, int32_t* status);

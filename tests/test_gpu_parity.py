@@ -208,3 +208,24 @@ def test_full_size_sampled_against_oracle(name, groups):
     err = np.abs(got[rows] - want[rows]).max()
     assert err <= gc.TOL, f"{name}: {err:.3e}"
     case.free()
+
+
+def test_staged_prefetch_comparator_matches_zero_copy():
+    """Copying the host pool into HBM first (the design the method argues against) gives the same answer."""
+    w = kvgen.LLAMA3_8B.replace(name="staged", batch=2, ctx=2100, seed=31)
+    case = gc.Case(w)
+    zero_copy = case.run()
+    blk = w.num_kv_heads * w.block_size * w.head_dim
+    ks = torch.empty(case.kv.host_split * blk, dtype=torch.int16, device="cuda")
+    vs = torch.empty_like(ks)
+    out = torch.full_like(case.q_dev, float("nan"))
+    case.attn.staged(case.q_dev, case.kv, out, ks, vs)
+    torch.cuda.synchronize()
+    assert case.attn.status() == 0
+    assert np.abs(out.cpu().numpy() - zero_copy).max() <= 1e-6
+    # the staging pool now holds a byte copy of the host pool
+    assert np.array_equal(ks.cpu().numpy().view(np.uint16), case.kv.k_host.array[:ks.numel()])
+    with pytest.raises(dkv.DkvError) as e:
+        case.attn.staged(case.q_dev, case.kv, out, None, None)
+    assert e.value.code == dkv.DKV_ERR_INVALID_ARG
+    case.free()
