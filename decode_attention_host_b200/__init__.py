@@ -39,7 +39,7 @@ DKV_PLACE_RANDOM = 1
 EXPORTED = ("dkv_create", "dkv_destroy", "dkv_attn_decode", "dkv_get_status", "dkv_last_error_string",
             "dkv_last_launch_count", "dkv_query_plan", "dkv_host_pool_alloc", "dkv_host_pool_free",
             "dkv_plan_blocks", "dkv_pack_kv", "dkv_profile_begin", "dkv_profile_end",
-            "dkv_attn_decode_noalloc", "dkv_plan_offload", "dkv_attn_decode_staged")
+            "dkv_attn_decode_noalloc", "dkv_plan_offload", "dkv_attn_decode_staged", "dkv_append_kv")
 
 
 class DkvConfig(ctypes.Structure):
@@ -80,6 +80,7 @@ def _load() -> ctypes.CDLL:
         "dkv_destroy": [vp],
         "dkv_attn_decode": [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32],
         "dkv_attn_decode_staged": [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, vp, vp],
+        "dkv_append_kv": [vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32],
         "dkv_get_status": [vp, c.POINTER(i32)],
         "dkv_last_error_string": [],
         "dkv_last_launch_count": [vp, c.POINTER(i32)],
@@ -144,6 +145,13 @@ def dkv_attn_decode_staged(h, q, k_host, v_host, k_dev, v_dev, block_table, seq_
     _check(lib.dkv_attn_decode_staged(h, _p(q), _p(k_host), _p(v_host), _p(k_dev), _p(v_dev), _p(block_table),
                                       _p(seq_lens), int(host_split), _p(out), stream, int(batch),
                                       int(block_table_stride), int(num_dev_blocks), _p(k_stage), _p(v_stage)))
+
+
+def dkv_append_kv(h, x, w_k, w_v, hidden, block_table, seq_lens, host_split, k_host, v_host, k_dev, v_dev, stream,
+                  batch, block_table_stride, num_dev_blocks) -> None:
+    _check(lib.dkv_append_kv(h, _p(x), _p(w_k), _p(w_v), int(hidden), _p(block_table), _p(seq_lens), int(host_split),
+                             _p(k_host), _p(v_host), _p(k_dev), _p(v_dev), stream, int(batch),
+                             int(block_table_stride), int(num_dev_blocks)))
 
 
 def dkv_get_status(h: int) -> int:
@@ -325,6 +333,16 @@ class DecodeAttention:
                                kv.k_dev if kv.num_dev_blocks else None, kv.v_dev if kv.num_dev_blocks else None,
                                kv.table_dev, kv.seq_lens_dev, kv.host_split, out, stream.cuda_stream, kv.batch,
                                kv.stride, kv.num_dev_blocks, k_stage, v_stage)
+
+    def append(self, x, w_k, w_v, kv: PagedKV, stream=None) -> None:
+        """Project x[B, hidden] with w_k, w_v [Hkv*D, hidden] and store at position seq_lens[b] of the cache."""
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(x.device)
+        dkv_append_kv(self.handle, x, w_k, w_v, x.shape[1], kv.table_dev, kv.seq_lens_dev, kv.host_split,
+                      kv.k_host.ptr or None, kv.v_host.ptr or None, kv.k_dev if kv.num_dev_blocks else None,
+                      kv.v_dev if kv.num_dev_blocks else None, stream.cuda_stream, kv.batch, kv.stride,
+                      kv.num_dev_blocks)
 
     def status(self) -> int:
         return dkv_get_status(self.handle)

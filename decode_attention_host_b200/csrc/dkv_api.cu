@@ -11,6 +11,7 @@
 
 #include "dkv.h"
 #include "dkv_error.h"
+#include "dkv_append.cuh"
 #include "dkv_kernels.cuh"
 
 namespace {
@@ -485,6 +486,66 @@ int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, const voi
                     int32_t num_dev_blocks) {
   return decode_impl(h, q, k_host, v_host, k_dev, v_dev, block_table, seq_lens, host_split, out, stream, batch,
                      block_table_stride, num_dev_blocks, nullptr, nullptr);
+}
+
+int dkv_append_kv(dkv_handle* h, const float* x, const void* w_k, const void* w_v, int32_t hidden,
+                  const int32_t* block_table, const int32_t* seq_lens, int32_t host_split, void* k_host,
+                  void* v_host, void* k_dev, void* v_dev, dkv_stream_t stream, int32_t batch,
+                  int32_t block_table_stride, int32_t num_dev_blocks) {
+  if (!h) return fail(DKV_ERR_INVALID_ARG, "dkv_append_kv: null handle");
+  const dkv_config& c = h->cfg;
+  if (batch < 0 || batch > c.max_batch) return fail(DKV_ERR_INVALID_ARG, "batch outside [0, max_batch]");
+  if (batch == 0) return DKV_OK;
+  if (!x || !w_k || !w_v || !block_table || !seq_lens) return fail(DKV_ERR_INVALID_ARG, "dkv_append_kv: null pointer");
+  if (hidden <= 0 || hidden % 8 != 0) return fail(DKV_ERR_INVALID_ARG, "hidden must be a positive multiple of 8");
+  if (block_table_stride < 1 || host_split < 0 || num_dev_blocks < 0 ||
+      static_cast<long long>(host_split) + num_dev_blocks > INT_MAX)
+    return fail(DKV_ERR_INVALID_ARG, "table stride / host_split / num_dev_blocks out of range");
+  if ((host_split > 0 && (!k_host || !v_host)) || (num_dev_blocks > 0 && (!k_dev || !v_dev)))
+    return fail(DKV_ERR_INVALID_ARG, "pool pointers are null");
+  auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+  if (mis16(x) || mis16(w_k) || mis16(w_v) || (host_split > 0 && (mis16(k_host) || mis16(v_host))) ||
+      (num_dev_blocks > 0 && (mis16(k_dev) || mis16(v_dev))))
+    return fail(DKV_ERR_INVALID_ARG, "x, weights and pools must be 16-byte aligned");
+  DeviceGuard guard(c.device);
+  if (!guard.ok) return fail(DKV_ERR_CUDA, "cudaSetDevice failed");
+  int rc;
+  if (host_split > 0) {
+    if ((rc = check_host_pool(h, k_host, 0)) != DKV_OK) return rc;
+    if ((rc = check_host_pool(h, v_host, 1)) != DKV_OK) return rc;
+  }
+  if (num_dev_blocks > 0) {
+    if ((rc = check_dev_pool(h, k_dev, 0)) != DKV_OK) return rc;
+    if ((rc = check_dev_pool(h, v_dev, 1)) != DKV_OK) return rc;
+  }
+  dkv::AppendParams ap{};
+  ap.x = x;
+  ap.w_k = static_cast<const uint16_t*>(w_k);
+  ap.w_v = static_cast<const uint16_t*>(w_v);
+  ap.table = block_table;
+  ap.seq_lens = seq_lens;
+  ap.k_host = static_cast<uint16_t*>(k_host);
+  ap.v_host = static_cast<uint16_t*>(v_host);
+  ap.k_dev = static_cast<uint16_t*>(k_dev);
+  ap.v_dev = static_cast<uint16_t*>(v_dev);
+  ap.status = h->status;
+  ap.batch = batch;
+  ap.hidden = hidden;
+  ap.hkv = c.num_kv_heads;
+  ap.head_dim = c.head_dim;
+  ap.block_size = c.block_size;
+  ap.stride = block_table_stride;
+  ap.host_split = host_split;
+  ap.num_dev_blocks = num_dev_blocks;
+  ap.max_len = (block_table_stride < c.max_blocks_per_seq ? block_table_stride : c.max_blocks_per_seq) * c.block_size;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(2 * c.num_kv_heads * c.head_dim / dkv::kAppendRows);
+  if (c.kv_dtype == DKV_KV_BF16)
+    dkv::append_kernel<true><<<grid, dkv::kAppendRows * 32, 0, s>>>(ap);
+  else
+    dkv::append_kernel<false><<<grid, dkv::kAppendRows * 32, 0, s>>>(ap);
+  DKV_CUDA(cudaGetLastError());
+  return DKV_OK;
 }
 
 int dkv_attn_decode_staged(dkv_handle* h, const float* q, const void* k_host, const void* v_host, const void* k_dev,

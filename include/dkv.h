@@ -141,6 +141,30 @@ DKV_API int dkv_attn_decode_staged(dkv_handle* h, const float* q, const void* k_
                                    int32_t batch, int32_t block_table_stride, int32_t num_dev_blocks, void* k_stage,
                                    void* v_stage);
 
+/*
+ * dkv_append_kv -- write side of the cache: project the new token of every
+ * sequence to K and V and store them, un-rotated, at its position (DirectKV
+ * README, opening summary: the fused kernel includes the K/V projection of new
+ * tokens; Step 6 checks K and V of "all new KV").
+ *   x           device fp32 [batch][hidden]: hidden state of the new token
+ *   w_k, w_v    device 16-bit (the handle's kv_dtype) [Hkv*D][hidden] row-major;
+ *               row h*D + d produces dim d of kv head h
+ *   hidden      > 0, multiple of 8; x, w_k, w_v and the pools 16-byte aligned
+ *   block_table, seq_lens, host_split, num_dev_blocks, pools: as for
+ *               dkv_attn_decode.  The new token goes to position L = seq_lens[b]
+ *               (the cache holds L tokens): block table entry L / S must name
+ *               its block, row L % S of that block is written.  seq_lens is not
+ *               changed; the caller advances it.
+ * k = W_k x and v = W_v x are accumulated in fp32 and rounded to the 16-bit
+ * type (nearest, ties to even).  Host-resident blocks are written through the
+ * mapped pointer.  Async on `stream`; positions beyond the table or ids
+ * outside both pools set DKV_STATUS_* bits and skip the store.
+ * Errors: INVALID_ARG, CUDA. */
+DKV_API int dkv_append_kv(dkv_handle* h, const float* x, const void* w_k, const void* w_v, int32_t hidden,
+                          const int32_t* block_table, const int32_t* seq_lens, int32_t host_split, void* k_host,
+                          void* v_host, void* k_dev, void* v_dev, dkv_stream_t stream, int32_t batch,
+                          int32_t block_table_stride, int32_t num_dev_blocks);
+
 /* dkv_get_status -- synchronise the handle's device, return the accumulated
  * DKV_STATUS_* bits in *status and clear them. */
 DKV_API int dkv_get_status(dkv_handle* h, int32_t* status);

@@ -55,6 +55,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
                                   c.c_void_p, c.c_void_p, c.c_int, c.c_double, c.c_double, c.c_void_p,
                                   c.c_void_p]
     lib.oracle_decode.restype = c.c_int
+    lib.oracle_project.argtypes = [c.c_int, c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_int, c.c_void_p]
+    lib.oracle_project.restype = c.c_int
     return lib
 
 
@@ -132,3 +134,18 @@ def decode(q: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, seq_lens: np.n
     if rc != 0:
         raise ValueError(f"oracle_decode failed with code {rc}")
     return out
+
+
+def project(x: np.ndarray, w_bits: np.ndarray, kv_dtype: int, lib=None) -> np.ndarray:
+    """y[b][r] = sum_h w[r][h] x[b][h] in fp64.  x float32 [B, H]; w uint16 [R, H]; returns float64 [B, R]."""
+    lib = lib or load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    w_bits = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    B, H = x.shape
+    R, H2 = w_bits.shape
+    assert H2 == H
+    y = np.empty((B, R), dtype=np.float64)
+    rc = lib.oracle_project(B, R, H, _ptr(x), _ptr(w_bits), int(kv_dtype), _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle_project failed with code {rc}")
+    return y

@@ -161,3 +161,26 @@ int oracle_decode(int B, int Hq, int Hkv, int D, int64_t Lmax, const float* q, c
   }
   return failed ? -2 : 0;
 }
+
+/*
+ * K/V projection of one new token per sequence (the write side of the cache).
+ *   DirectKV README, opening summary: the fused kernel includes the K/V
+ *   projection of the new token; Step 6 reports K and V errors for "all new
+ *   KV".  The projection is a plain matrix-vector product per sequence:
+ *     y[b][r] = sum_h w[r][h] * x[b][h]
+ *   x    [B][H]  fp32
+ *   w    [R][H]  raw 16-bit (kv_dtype), row r = kv head r / D, dim r % D
+ *   y    [B][R]  fp64 (exact products, fp64 sums)
+ */
+int oracle_project(int B, int R, int H, const float* x, const uint16_t* w, int kv_dtype, double* y) {
+  if (B < 0 || R < 0 || H < 0) return -1;
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < R; ++r) {
+    for (int b = 0; b < B; ++b) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h) acc += decode16(w[(size_t)r * H + h], kv_dtype) * (double)x[(size_t)b * H + h];
+      y[(size_t)b * R + r] = acc;
+    }
+  }
+  return 0;
+}

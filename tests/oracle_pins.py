@@ -237,7 +237,22 @@ def pin_explicit_scale(lib):
     assert np.abs(c - want).max() < 1e-12
 
 
+def pin_projection(lib):
+    """The K/V projection equals numpy's matmul of the widened weights; one-hot x picks a weight column."""
+    rng = np.random.default_rng(12)
+    for dt, B, R, H in ((BF16, 3, 40, 96), (F16, 2, 17, 64)):
+        x = rng.standard_normal((B, H)).astype(np.float32)
+        conv = kvgen.f32_to_bf16_bits if dt == BF16 else kvgen.f32_to_f16_bits
+        w = conv(rng.standard_normal((R, H)).astype(np.float32))
+        got = oracle.project(x, w, dt, lib=lib)
+        want = x.astype(np.float64) @ _widen(w, dt).T
+        assert np.abs(got - want).max() < 1e-12
+        e = np.zeros((1, H), np.float32)
+        e[0, 5] = 1.0
+        assert np.array_equal(oracle.project(e, w, dt, lib=lib)[0], _widen(w, dt)[:, 5])
+
+
 ALL_PINS = [pin_f16_decode_exhaustive, pin_bf16_decode_exhaustive, pin_rope_closed_forms, pin_rope_vs_complex,
             pin_rope_vs_hf, pin_rope_invariants, pin_attention_vs_numpy, pin_attention_vs_torch_hf,
             pin_special_cases, pin_dominant_key, pin_gqa_equals_repeated_mha, pin_ignores_tokens_past_length,
-            pin_linear_in_v, pin_explicit_scale]
+            pin_linear_in_v, pin_explicit_scale, pin_projection]

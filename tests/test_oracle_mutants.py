@@ -28,6 +28,8 @@ MUTANTS = {
     "bf16_wrong_shift": ("uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)b) << 15;"),
     "v_read_from_k": ("o[d] += w * decode16(vb[(size_t)t * D + d], kv_dtype);",
                       "o[d] += w * decode16(kb[(size_t)t * D + d], kv_dtype);"),
+    "projection_transposed": ("decode16(w[(size_t)r * H + h], kv_dtype) * (double)x[(size_t)b * H + h]",
+                              "decode16(w[(size_t)h * R + r], kv_dtype) * (double)x[(size_t)b * H + h]"),
     "last_token_dropped": ("for (int64_t t = 0; t < L; ++t) {\n        double w", "for (int64_t t = 0; t + 1 < L; ++t) {\n        double w"),
 }
 
