@@ -47,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("dkv", "reference"), default="dkv")
     ap.add_argument("--mode", choices=("zero_copy", "staged"), default="zero_copy",
                     help="staged: the prefetch comparator (host pool copied into HBM each step)")
+    ap.add_argument("--queries", type=int, default=1,
+                    help="query tokens per sequence (>1: multi-token queries, e.g. speculative verification)")
     ap.add_argument("--host-ctas", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -263,11 +265,15 @@ def run_dkv(args):
     lens = kvgen.gen_seq_lens(w)
     k, v = kvgen.gen_kv(w, lens)
     placement = dkv.DKV_PLACE_PREFIX_HOST if w.placement == "prefix_host" else dkv.DKV_PLACE_RANDOM
+    tq = args.queries
+    # multi-token queries: the cache holds L + tq - 1 tokens, query i sits at position L + i
     kv = dkv.PagedKV(k, v, lens, w.block_size, placement, w.host_fraction, w.shuffle, w.seed, device=local)
+    if tq > 1:
+        kv.seq_lens_dev.copy_(torch.from_numpy(lens - (tq - 1)))
     attn = dkv.DecodeAttention(w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
                                dkv.DKV_KV_BF16 if w.kv_dtype == kvgen.BF16 else dkv.DKV_KV_F16, w.rope_base,
-                               w.batch, kv.stride, device=local, host_ctas=args.host_ctas)
-    keep_logical = rank == 0 and world == 1 and not args.no_cpu_baseline
+                               w.batch * tq, kv.stride, device=local, host_ctas=args.host_ctas)
+    keep_logical = rank == 0 and world == 1 and not args.no_cpu_baseline and args.queries == 1
     if not keep_logical:
         del k, v
     q_dev = torch.from_numpy(q).to(device)
@@ -275,6 +281,10 @@ def run_dkv(args):
     stream = torch.cuda.current_stream(device)
     b_pcie = measure_pcie_gbs(device)
 
+    if tq > 1:
+        q_dev = torch.from_numpy(np.random.default_rng(w.seed).standard_normal(
+            (w.batch, tq, w.num_q_heads, w.head_dim)).astype(np.float32)).to(device)
+        out = torch.empty_like(q_dev)
     if args.mode == "staged":
         blk = w.num_kv_heads * w.block_size * w.head_dim
         k_stage = torch.empty(max(1, kv.host_split * blk), dtype=torch.int16, device=device)
@@ -282,6 +292,9 @@ def run_dkv(args):
 
         def step():
             attn.staged(q_dev, kv, out, k_stage, v_stage, stream)
+    elif tq > 1:
+        def step():
+            attn.multi(q_dev, kv, out, stream)
     else:
         def step():
             attn(q_dev, kv, out, stream)
@@ -314,8 +327,8 @@ def run_dkv(args):
     # ---- end to end through the public API: inputs from pinned host memory, result back to the host
     e2e = None
     if not args.no_e2e:
-        q_h = torch.from_numpy(q).pin_memory()
-        lens_h = torch.from_numpy(kv.seq_lens).pin_memory()
+        q_h = q_dev.cpu().pin_memory()
+        lens_h = torch.from_numpy(kv.seq_lens - (tq - 1)).pin_memory()   # base lengths L
         table_h = torch.from_numpy(kv.table).pin_memory()
         out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         h2d = q_h.numel() * 4 + lens_h.numel() * 4 + table_h.numel() * 4
@@ -401,6 +414,7 @@ def run_dkv(args):
         "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
         "config": dict(workload_config(w, world), host_bytes=host_bytes, dev_bytes=dev_bytes, mode=args.mode,
+                       query_tokens=tq,
                        l2="inputs larger than L2: %.0f MiB of KV per step vs 126 MB L2" % ((host_bytes + dev_bytes) / 2**20)),
         "roofline": ({k2: dominant[k2] for k2 in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
                      if dominant else None),

@@ -39,7 +39,8 @@ DKV_PLACE_RANDOM = 1
 EXPORTED = ("dkv_create", "dkv_destroy", "dkv_attn_decode", "dkv_get_status", "dkv_last_error_string",
             "dkv_last_launch_count", "dkv_query_plan", "dkv_host_pool_alloc", "dkv_host_pool_free",
             "dkv_plan_blocks", "dkv_pack_kv", "dkv_profile_begin", "dkv_profile_end",
-            "dkv_attn_decode_noalloc", "dkv_plan_offload", "dkv_attn_decode_staged", "dkv_append_kv")
+            "dkv_attn_decode_noalloc", "dkv_plan_offload", "dkv_attn_decode_staged", "dkv_append_kv",
+            "dkv_attn_decode_multi")
 
 
 class DkvConfig(ctypes.Structure):
@@ -81,6 +82,7 @@ def _load() -> ctypes.CDLL:
         "dkv_attn_decode": [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32],
         "dkv_attn_decode_staged": [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, vp, vp],
         "dkv_append_kv": [vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32],
+        "dkv_attn_decode_multi": [vp, i32, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32],
         "dkv_get_status": [vp, c.POINTER(i32)],
         "dkv_last_error_string": [],
         "dkv_last_launch_count": [vp, c.POINTER(i32)],
@@ -152,6 +154,13 @@ def dkv_append_kv(h, x, w_k, w_v, hidden, block_table, seq_lens, host_split, k_h
     _check(lib.dkv_append_kv(h, _p(x), _p(w_k), _p(w_v), int(hidden), _p(block_table), _p(seq_lens), int(host_split),
                              _p(k_host), _p(v_host), _p(k_dev), _p(v_dev), stream, int(batch),
                              int(block_table_stride), int(num_dev_blocks)))
+
+
+def dkv_attn_decode_multi(h, num_queries, q, k_host, v_host, k_dev, v_dev, block_table, seq_lens, host_split, out,
+                          stream, batch, block_table_stride, num_dev_blocks) -> None:
+    _check(lib.dkv_attn_decode_multi(h, int(num_queries), _p(q), _p(k_host), _p(v_host), _p(k_dev), _p(v_dev),
+                                     _p(block_table), _p(seq_lens), int(host_split), _p(out), stream, int(batch),
+                                     int(block_table_stride), int(num_dev_blocks)))
 
 
 def dkv_get_status(h: int) -> int:
@@ -343,6 +352,16 @@ class DecodeAttention:
                       kv.k_host.ptr or None, kv.v_host.ptr or None, kv.k_dev if kv.num_dev_blocks else None,
                       kv.v_dev if kv.num_dev_blocks else None, stream.cuda_stream, kv.batch, kv.stride,
                       kv.num_dev_blocks)
+
+    def multi(self, q, kv: PagedKV, out, stream=None) -> None:
+        """q, out [B, Tq, Hq, D]: query i of sequence b at position seq_lens[b] + i, causal over the cache."""
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(q.device)
+        dkv_attn_decode_multi(self.handle, q.shape[1], q, kv.k_host.ptr or None, kv.v_host.ptr or None,
+                              kv.k_dev if kv.num_dev_blocks else None, kv.v_dev if kv.num_dev_blocks else None,
+                              kv.table_dev, kv.seq_lens_dev, kv.host_split, out, stream.cuda_stream, kv.batch,
+                              kv.stride, kv.num_dev_blocks)
 
     def status(self) -> int:
         return dkv_get_status(self.handle)

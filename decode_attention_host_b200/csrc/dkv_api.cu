@@ -13,6 +13,7 @@
 #include "dkv_error.h"
 #include "dkv_append.cuh"
 #include "dkv_kernels.cuh"
+#include "dkv_multi.cuh"
 
 namespace {
 
@@ -101,6 +102,24 @@ SplitEntry pick_split(int D, int G, bool bf16, bool rope) {
   return rope ? pick_split_rope<NST, true>(D, G, bf16) : pick_split_rope<NST, false>(D, G, bf16);
 }
 
+template <int D, bool BF16, bool ROPE>
+void launch_multi(dim3 grid, size_t smem, cudaStream_t s, const dkv::SplitParams& p) {
+  dkv::multi_kernel<D, BF16, ROPE><<<grid, dkv::kThreads, smem, s>>>(p);
+}
+
+SplitEntry pick_multi(int D, bool bf16, bool rope) {
+#define DKV_MCASE(DD, BB, RR) \
+  if (D == DD && bf16 == BB && rope == RR) \
+    return {&launch_multi<DD, BB, RR>, reinterpret_cast<const void*>(&dkv::multi_kernel<DD, BB, RR>)};
+  DKV_MCASE(64, false, false) DKV_MCASE(64, false, true) DKV_MCASE(64, true, false) DKV_MCASE(64, true, true)
+  DKV_MCASE(128, false, false) DKV_MCASE(128, false, true) DKV_MCASE(128, true, false) DKV_MCASE(128, true, true)
+#undef DKV_MCASE
+  return {nullptr, nullptr};
+}
+
+// shared memory of the multi-token kernel: per warp a 2-stage (K, V) ring and one rotated-K lo tile
+size_t multi_smem(int D) { return static_cast<size_t>(dkv::kWarps) * 5 * dkv::kTileTokens * D * 2; }
+
 using MergeFn = void (*)(dim3, size_t, cudaStream_t, const dkv::MergeParams&);
 template <int D, int NG>
 void launch_merge(dim3 grid, size_t smem, cudaStream_t s, const dkv::MergeParams& p) {
@@ -124,7 +143,7 @@ struct dkv_handle {
   cudaStream_t aux = nullptr;
   cudaEvent_t ev_fork = nullptr;
   cudaEvent_t ev_join = nullptr;
-  SplitEntry host_kernel{}, dev_kernel{};
+  SplitEntry host_kernel{}, dev_kernel{}, multi_kernel{};
   MergeFn merge = nullptr;
   const void* ok_host[2] = {nullptr, nullptr};
   const void* ok_dev[4] = {nullptr, nullptr, nullptr, nullptr};
@@ -171,14 +190,14 @@ void release(dkv_handle* h) {
   delete h;
 }
 
-void plan_splits(const dkv_handle* h, int batch, int stride, int* nsplit, int* bps) {
+void plan_splits(const dkv_handle* h, int batch, int stride, int* nsplit, int* bps, int num_queries = 1) {
   const int nblk = stride < h->cfg.max_blocks_per_seq ? stride : h->cfg.max_blocks_per_seq;
   if (nblk <= 0 || batch <= 0) {
     *nsplit = 1;
     *bps = 1;
     return;
   }
-  const long per = static_cast<long>(batch) * h->cfg.num_kv_heads;
+  const long per = static_cast<long>(batch) * num_queries * h->cfg.num_kv_heads;
   const int target = static_cast<int>((h->units_target + per - 1) / per) > 0
                          ? static_cast<int>((h->units_target + per - 1) / per)
                          : 1;
@@ -261,6 +280,7 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   const bool rope = c.rope_base > 0.0;
   h->host_kernel = pick_split<kHostStages>(c.head_dim, G, bf16, rope);
   h->dev_kernel = pick_split<kDevStages>(c.head_dim, G, bf16, rope);
+  h->multi_kernel = pick_multi(c.head_dim, bf16, c.rope_base > 0.0);
   h->merge = c.head_dim == 64 ? &launch_merge<64, 16> : &launch_merge<128, 8>;
 
   auto bail = [&](int code) {
@@ -277,6 +297,9 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   e = cudaFuncSetAttribute(h->dev_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(split_smem(c.head_dim, kDevStages)));
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(HBM kernel)"));
+  e = cudaFuncSetAttribute(h->multi_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(multi_smem(c.head_dim)));
+  if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(multi-token kernel)"));
   if (cudaMalloc(&h->part_o, h->part_rows * c.head_dim * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&h->part_lse, h->part_rows * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&h->status, sizeof(int32_t)) != cudaSuccess ||
@@ -338,8 +361,13 @@ namespace {
 int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v_host, const void* k_dev,
                 const void* v_dev, const int32_t* block_table, const int32_t* seq_lens, int32_t host_split, float* out,
                 dkv_stream_t stream, int32_t batch, int32_t block_table_stride, int32_t num_dev_blocks, void* k_stage,
-                void* v_stage) {
+                void* v_stage, int32_t num_queries = 0) {
   const bool staged = k_stage != nullptr || v_stage != nullptr;
+  const bool multi = num_queries > 0;  // the multi-token kernel (num_queries >= 1 query tokens per sequence)
+  const int nq = multi ? num_queries : 1;
+  if (multi && (h == nullptr || num_queries * (h->cfg.num_q_heads / h->cfg.num_kv_heads) > dkv::kMultiMaxRows ||
+                static_cast<long long>(batch) * num_queries > h->cfg.max_batch))
+    return fail(DKV_ERR_INVALID_ARG, "num_queries * group size must be <= 16 and batch * num_queries <= max_batch");
   if (!h) return fail(DKV_ERR_INVALID_ARG, "dkv_attn_decode: null handle");
   if (batch < 0 || batch > h->cfg.max_batch) return fail(DKV_ERR_INVALID_ARG, "batch outside [0, max_batch]");
   if (batch == 0) {
@@ -379,9 +407,9 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
 
   const dkv_config& c = h->cfg;
   int nsplit, bps;
-  plan_splits(h, batch, block_table_stride, &nsplit, &bps);
+  plan_splits(h, batch, block_table_stride, &nsplit, &bps, nq);
   const int nslots = 2 * nsplit;
-  if (static_cast<size_t>(batch) * c.num_q_heads * nslots > h->part_rows)
+  if (static_cast<size_t>(batch) * nq * c.num_q_heads * nslots > h->part_rows)
     return fail(DKV_ERR_INVALID_ARG, "internal: split plan exceeds the workspace");
   const int n_units = batch * nsplit * c.num_kv_heads;
   const int nblk_cap = block_table_stride < c.max_blocks_per_seq ? block_table_stride : c.max_blocks_per_seq;
@@ -406,6 +434,12 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   sp.n_units = n_units;
   sp.rope = c.rope_base > 0.0 ? 1 : 0;
   sp.qscale = h->qscale;
+  sp.extra_tokens = nq - 1;
+  sp.num_queries = nq;
+  const SplitEntry& host_k = multi ? h->multi_kernel : h->host_kernel;
+  const SplitEntry& dev_k = multi ? h->multi_kernel : h->dev_kernel;
+  const size_t host_smem = multi ? multi_smem(c.head_dim) : split_smem(c.head_dim, kHostStages);
+  const size_t dev_smem = multi ? multi_smem(c.head_dim) : split_smem(c.head_dim, kDevStages);
 
   const int unit_ctas = (n_units + dkv::kWarps - 1) / dkv::kWarps;
   int launches = 0;
@@ -423,7 +457,7 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
     hp.id_hi = host_split;
     hp.slot_base = 0;
     const int dev_ctas = unit_ctas < 2 * h->sm_count ? unit_ctas : 2 * h->sm_count;
-    h->dev_kernel.fn(dim3(dev_ctas), split_smem(c.head_dim, kDevStages), s, hp);
+    dev_k.fn(dim3(dev_ctas), dev_smem, s, hp);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 0, s, true)) != DKV_OK) return rc;
     ++launches;
@@ -438,7 +472,7 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
     hp.slot_base = 0;
     const int grid = unit_ctas < h->host_ctas ? unit_ctas : h->host_ctas;
     if ((rc = prof_mark(h, 0, h->aux, false)) != DKV_OK) return rc;
-    h->host_kernel.fn(dim3(grid), split_smem(c.head_dim, kHostStages), h->aux, hp);
+    host_k.fn(dim3(grid), host_smem, h->aux, hp);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 0, h->aux, true)) != DKV_OK) return rc;
     DKV_CUDA(cudaEventRecord(h->ev_join, h->aux));
@@ -453,7 +487,7 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
     dp.slot_base = nsplit;
     if ((rc = prof_mark(h, 1, s, false)) != DKV_OK) return rc;
     const int dev_ctas = unit_ctas < 2 * h->sm_count ? unit_ctas : 2 * h->sm_count;  // one resident wave
-    h->dev_kernel.fn(dim3(dev_ctas), split_smem(c.head_dim, kDevStages), s, dp);
+    dev_k.fn(dim3(dev_ctas), dev_smem, s, dp);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 1, s, true)) != DKV_OK) return rc;
     ++launches;
@@ -468,7 +502,7 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   mp.has_host = host_split > 0;
   mp.has_dev = num_dev_blocks > 0;
   if ((rc = prof_mark(h, 2, s, false)) != DKV_OK) return rc;
-  h->merge(dim3(batch * c.num_q_heads), nslots * sizeof(float), s, mp);
+  h->merge(dim3(batch * nq * c.num_q_heads), nslots * sizeof(float), s, mp);
   DKV_CUDA(cudaGetLastError());
   if ((rc = prof_mark(h, 2, s, true)) != DKV_OK) return rc;
   ++launches;
@@ -546,6 +580,15 @@ int dkv_append_kv(dkv_handle* h, const float* x, const void* w_k, const void* w_
     dkv::append_kernel<false><<<grid, dkv::kAppendRows * 32, 0, s>>>(ap);
   DKV_CUDA(cudaGetLastError());
   return DKV_OK;
+}
+
+int dkv_attn_decode_multi(dkv_handle* h, int32_t num_queries, const float* q, const void* k_host, const void* v_host,
+                          const void* k_dev, const void* v_dev, const int32_t* block_table, const int32_t* seq_lens,
+                          int32_t host_split, float* out, dkv_stream_t stream, int32_t batch,
+                          int32_t block_table_stride, int32_t num_dev_blocks) {
+  if (!h || num_queries < 1) return fail(DKV_ERR_INVALID_ARG, "dkv_attn_decode_multi: null handle or num_queries < 1");
+  return decode_impl(h, q, k_host, v_host, k_dev, v_dev, block_table, seq_lens, host_split, out, stream, batch,
+                     block_table_stride, num_dev_blocks, nullptr, nullptr, num_queries);
 }
 
 int dkv_attn_decode_staged(dkv_handle* h, const float* q, const void* k_host, const void* v_host, const void* k_dev,

@@ -69,6 +69,8 @@ struct SplitParams {
   int32_t n_units;          // B * nsplit * Hkv
   int32_t rope;             // 0: no rotation
   float qscale;             // softmax scale * log2(e)
+  int32_t extra_tokens;     // tokens past seq_lens that belong to the unit (multi-token queries: Tq - 1)
+  int32_t num_queries;      // query tokens per sequence (1 for decode)
 };
 
 struct MergeParams {
@@ -163,6 +165,29 @@ __device__ __forceinline__ void ldsm_x4_t(const void* p, uint32_t& r0, uint32_t&
                : "r"(smem_u32(p)));
 }
 
+// Four 8x8 b16 matrices from shared memory (mma B operand of a row-major [n][k] tile).
+__device__ __forceinline__ void ldsm_x4(const void* p, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
+}
+
+// D(16x8,f32) += A(16x16) * B(16x8) with all four C rows live.
+template <bool BF16>
+__device__ __forceinline__ void mma16816_full(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (BF16) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};\n"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};\n"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
 // D(16x8,f32) += A(16x16) * B(16x8), A and B both bf16 or both fp16, for A
 // whose rows 8..15 are zero: only the C/D rows 0..7 (c[0], c[1]) are kept; the
 // rows 8..15 take a zero input and their outputs are discarded, so they cost
@@ -217,7 +242,8 @@ struct TileStream {
     const int c = bc % p.nsplit;
     b = bc / p.nsplit;
     L = p.seq_lens[b];
-    bad_len = (L < 0 || L > p.max_len);
+    bad_len = (L < 0 || L + p.extra_tokens > p.max_len);
+    L += p.extra_tokens;
     const int nblk = bad_len ? 0 : (L + p.block_size - 1) / p.block_size;
     j = c * p.bps;
     j_end = min(j + p.bps, nblk);

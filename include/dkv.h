@@ -123,6 +123,26 @@ DKV_API int dkv_attn_decode(dkv_handle* h, const float* q, const void* k_host, c
                     int32_t batch, int32_t block_table_stride, int32_t num_dev_blocks);
 
 /*
+ * dkv_attn_decode_multi -- num_queries (Tq) query tokens per sequence over the
+ * same split cache, for speculative verification or chunked prefill (the
+ * pages' CUDA test runs a "Prefill (all new KV)" case, DirectKV README,
+ * Step 6).  Query i of sequence b sits at position L_b + i and attends to the
+ * cached tokens t < L_b + i, so the cache must already hold the tokens
+ * L_b .. L_b + Tq - 2 (see dkv_append_kv) and the table must cover them.
+ * Tq = 1 computes exactly what dkv_attn_decode computes.
+ *   q    device fp32 [batch][Tq][Hq][D]        out  device fp32 [batch][Tq][Hq][D]
+ *   Tq * (Hq / Hkv) <= 16 and batch * Tq <= max_batch; the rest as for
+ *   dkv_attn_decode (L_b + Tq - 1 <= table capacity, else status + NaN rows).
+ * Both contractions run on the tensor cores (mma.sync, with 16-bit hi + lo
+ * splits of the rotated keys, the queries and the softmax weights).
+ * Errors: as dkv_attn_decode. */
+DKV_API int dkv_attn_decode_multi(dkv_handle* h, int32_t num_queries, const float* q, const void* k_host,
+                                  const void* v_host, const void* k_dev, const void* v_dev,
+                                  const int32_t* block_table, const int32_t* seq_lens, int32_t host_split,
+                                  float* out, dkv_stream_t stream, int32_t batch, int32_t block_table_stride,
+                                  int32_t num_dev_blocks);
+
+/*
  * dkv_attn_decode_staged -- the staged-prefetch comparator: the design the
  * zero-copy method is measured against (SplitKernel README, Overview:
  * prefetch-based offloading that first moves offloaded data back into HBM;

@@ -40,7 +40,7 @@ class Case:
     """Inputs of one workload, its paged cache and the CUDA output."""
 
     def __init__(self, w: kvgen.Workload, lens=None, host_fraction=None, placement=None, shuffle=None,
-                 plan_seed=None, stride=None, host_ctas=0):
+                 plan_seed=None, stride=None, host_ctas=0, max_batch=None):
         self.w = w
         self.q = kvgen.gen_q(w)
         self.lens = kvgen.gen_seq_lens(w) if lens is None else np.asarray(lens, dtype=np.int32)
@@ -50,7 +50,8 @@ class Case:
                               w.host_fraction if host_fraction is None else host_fraction,
                               w.shuffle if shuffle is None else shuffle,
                               w.seed if plan_seed is None else plan_seed, stride=stride)
-        self.attn = attention_for(w, max_blocks=max(w.max_blocks_per_seq(), self.kv.stride), host_ctas=host_ctas)
+        self.attn = attention_for(w, max_blocks=max(w.max_blocks_per_seq(), self.kv.stride), host_ctas=host_ctas,
+                                  max_batch=max_batch)
         self.q_dev = torch.from_numpy(self.q).cuda()
         self.out = torch.full_like(self.q_dev, float("nan"))
 
