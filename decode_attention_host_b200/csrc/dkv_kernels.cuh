@@ -31,12 +31,12 @@
 // keeps its own online-softmax state (running max, sum, un-normalised
 // output) over its tokens, and the four states are merged once per unit.
 //
-// RoPE.  theta_i(p) = p * base^(-2i/D).  The angle at the first token of a
-// tile is formed in fp64 and reduced modulo 2*pi before the fp32 sin/cos, so
-// positions up to 2^24 keep full accuracy; the three later tokens of the same
-// lane follow by multiplying with exp(i*4*theta_i(1)) (exact-to-fp32 step,
-// error growth < 1e-6 over a tile).  Scores carry scale*log2(e) so the
-// softmax works with exp2.
+// RoPE.  theta_i(p) = p * base^(-2i/D).  A seed angle is formed in fp64 and
+// reduced modulo 2*pi before the fp32 sin/cos, so positions up to 2^24 keep
+// full accuracy; the later tokens of a lane follow by multiplying with
+// exp(i*4*theta_i(1)), across tiles too while positions continue, with a
+// fresh seed at least every 8 tiles (at most 32 fp32 steps, error ~4e-6).
+// Scores carry scale*log2(e) so the softmax works with exp2.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -493,24 +493,22 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const char* sk = ring + static_cast<size_t>(slot) * 2 * TILE;
     const char* sv = sk + TILE;
     const int nvalid = d.meta & 0xff;
-    // ---- scores: rotate K rows on the fly (CUDA cores, fp32 pairs)
-    float2 C[NP2], S[NP2], NS[NP2];
+    // ---- scores: rotate K rows on the fly (CUDA cores, fp32 pairs).  The
+    // rotation state (Cc, Sc, NSc) carries over when this tile continues the
+    // previous one; a fresh fp64-reduced seed at least every 8 tiles.
     if constexpr (ROPE) {
-      if (d.p0 == next_pos && chain < 4) {
-#pragma unroll
-        for (int j = 0; j < NP2; ++j) {
-          C[j] = Cc[j];
-          S[j] = Sc[j];
-          NS[j] = NSc[j];
-        }
+      if (d.p0 == next_pos && chain < 8) {
         ++chain;
       } else {
-        seeds(d.p0 + tg, C, S);
+        seeds(d.p0 + tg, Cc, Sc);
 #pragma unroll
-        for (int j = 0; j < NP2; ++j) NS[j] = make_float2(-S[j].x, -S[j].y);
+        for (int j = 0; j < NP2; ++j) NSc[j] = make_float2(-Sc[j].x, -Sc[j].y);
         chain = 1;
       }
     }
+    float2 (&C)[NP2] = Cc;
+    float2 (&S)[NP2] = Sc;
+    float2 (&NS)[NP2] = NSc;
     float v[4 * G];  // partial scores, index g * 4 + m
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -548,15 +546,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
         v[g * 4 + m] = a.x + a.y;
       }
     }
-    if constexpr (ROPE) {
-#pragma unroll
-      for (int j = 0; j < NP2; ++j) {
-        Cc[j] = C[j];
-        Sc[j] = S[j];
-        NSc[j] = NS[j];
-      }
-      next_pos = d.p0 + kTileTokens;
-    }
+    if constexpr (ROPE) next_pos = d.p0 + kTileTokens;
     // ---- reduce-scatter over the 8 lanes of the token group: halve the value
     // set at each xor step; lane li ends with scores g*4+m = li*(4G/8) + k
     constexpr int NV = 4 * G;
