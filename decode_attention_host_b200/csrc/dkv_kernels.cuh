@@ -26,16 +26,17 @@
 // Lane layout inside a warp.  8 lanes share one token: lane li (0..7) of
 // token group tg (0..3) owns the NeoX pairs i in [li*PPL, li*PPL+PPL),
 // i.e. dims i and i + D/2 (PPL = D/16).  The 16 tokens of a tile are split
-// tg, tg+4, tg+8, tg+12 over the four token groups.  Scores are reduced over
-// the 8 lanes of a token group with three xor-shuffles; each token group
-// keeps its own online-softmax state (running max, sum, un-normalised
-// output) over its tokens, and the four states are merged once per unit.
+// tg, tg+4, tg+8, tg+12 over the four token groups.  The partial scores of
+// the 8 lanes of a token group are combined by a three-step xor
+// reduce-scatter, after which each lane owns the scores of one query head;
+// the online softmax keeps one running max and sum per head, and the
+// softmax weights drive the PV product on the tensor cores.
 //
 // RoPE.  theta_i(p) = p * base^(-2i/D).  A seed angle is formed in fp64 and
 // reduced modulo 2*pi before the fp32 sin/cos, so positions up to 2^24 keep
 // full accuracy; the later tokens of a lane follow by multiplying with
 // exp(i*4*theta_i(1)), across tiles too while positions continue, with a
-// fresh seed at least every 8 tiles (at most 32 fp32 steps, error ~4e-6).
+// fresh seed at least every 16 tiles (at most 64 fp32 steps, error ~1e-5).
 // Scores carry scale*log2(e) so the softmax works with exp2.
 #pragma once
 
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   extern __shared__ __align__(128) char smem[];
   __shared__ TileDesc meta[kWarps][NST];
   __shared__ double s_freq[PPL][8];            // [r][li]: base^(-2i/D), i = li*PPL + r
-  __shared__ float2 s_e[NP2][8], s_f[NP2][8], s_nf[NP2][8];  // 4-token step: cos, sin, -sin (pairs)
+  __shared__ float2 s_e[NP2][8], s_f[NP2][8];  // 4-token step: cos, sin (pairs)
   __shared__ __align__(16) float s_p[kWarps][4][4][4];  // softmax weights of the tile: [head][token group][m]
 
   const int warp = threadIdx.x >> 5;
@@ -334,12 +335,18 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     rope_cs(4, w, c, sn);
     float* e = reinterpret_cast<float*>(&s_e[r >> 1][l]) + (r & 1);
     float* f = reinterpret_cast<float*>(&s_f[r >> 1][l]) + (r & 1);
-    float* nf = reinterpret_cast<float*>(&s_nf[r >> 1][l]) + (r & 1);
     *e = c;
     *f = sn;
-    *nf = -sn;
   }
   __syncthreads();
+
+  // 4-position step factors of this lane's pairs, kept in registers
+  float2 re[NP2], rf[NP2];
+#pragma unroll
+  for (int j = 0; j < NP2; ++j) {
+    re[j] = s_e[j][li];
+    rf[j] = s_f[j][li];
+  }
 
   TileStream ts;
   ts.unit = blockIdx.x * kWarps + warp;
@@ -398,7 +405,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   bool poisoned = false;
   int cur = -1;
   // RoPE factors carried from one tile to the next when positions continue
-  float2 Cc[NP2], Sc[NP2], NSc[NP2];
+  float2 Cc[NP2], Sc[NP2];
   int next_pos = -1, chain = 0;
 
   auto seeds = [&](int pos, float2 (&C)[NP2], float2 (&S)[NP2]) {
@@ -494,21 +501,18 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const char* sv = sk + TILE;
     const int nvalid = d.meta & 0xff;
     // ---- scores: rotate K rows on the fly (CUDA cores, fp32 pairs).  The
-    // rotation state (Cc, Sc, NSc) carries over when this tile continues the
-    // previous one; a fresh fp64-reduced seed at least every 8 tiles.
+    // rotation state (Cc, Sc) carries over when this tile continues the
+    // previous one; a fresh fp64-reduced seed at least every 16 tiles.
     if constexpr (ROPE) {
-      if (d.p0 == next_pos && chain < 8) {
+      if (d.p0 == next_pos && chain < 16) {
         ++chain;
       } else {
         seeds(d.p0 + tg, Cc, Sc);
-#pragma unroll
-        for (int j = 0; j < NP2; ++j) NSc[j] = make_float2(-Sc[j].x, -Sc[j].y);
         chain = 1;
       }
     }
     float2 (&C)[NP2] = Cc;
     float2 (&S)[NP2] = Sc;
-    float2 (&NS)[NP2] = NSc;
     float v[4 * G];  // partial scores, index g * 4 + m
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -521,28 +525,24 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
 #pragma unroll
         for (int j = 0; j < NP2; ++j) {
           const float2 x = X[j], y = Y[j];
-          X[j] = __ffma2_rn(y, NS[j], __fmul2_rn(x, C[j]));   // x c - y s
+          const float2 ns = __fmul2_rn(S[j], make_float2(-1.f, -1.f));
+          X[j] = __ffma2_rn(y, ns, __fmul2_rn(x, C[j]));      // x c - y s
           Y[j] = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));    // y c + x s
           // advance 4 positions: (C + iS)(E + iF); after m = 3 this is the
           // first token of the tile 16 positions on
-          const float2 e = s_e[j][li], f = s_f[j][li], nf = s_nf[j][li];
-          const float2 cn = __ffma2_rn(NS[j], f, __fmul2_rn(C[j], e));
-          const float2 sn = __ffma2_rn(C[j], f, __fmul2_rn(S[j], e));
-          NS[j] = __ffma2_rn(C[j], nf, __fmul2_rn(NS[j], e));
+          const float2 cn = __ffma2_rn(ns, rf[j], __fmul2_rn(C[j], re[j]));
+          S[j] = __ffma2_rn(C[j], rf[j], __fmul2_rn(S[j], re[j]));
           C[j] = cn;
-          S[j] = sn;
         }
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float2 ax = __fmul2_rn(QX[g][0], X[0]);
-        float2 ay = __fmul2_rn(QY[g][0], Y[0]);
+        float2 a = __ffma2_rn(QY[g][0], Y[0], __fmul2_rn(QX[g][0], X[0]));
 #pragma unroll
         for (int j = 1; j < NP2; ++j) {
-          ax = __ffma2_rn(QX[g][j], X[j], ax);
-          ay = __ffma2_rn(QY[g][j], Y[j], ay);
+          a = __ffma2_rn(QX[g][j], X[j], a);
+          a = __ffma2_rn(QY[g][j], Y[j], a);
         }
-        const float2 a = __fadd2_rn(ax, ay);
         v[g * 4 + m] = a.x + a.y;
       }
     }
