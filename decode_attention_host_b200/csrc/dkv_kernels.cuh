@@ -52,6 +52,8 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kFlagPoison = 1 << 8;
+constexpr int kSubShift = 9;                   // tile index inside its block (block_size <= 1024)
+constexpr int kSubMask = 63;
 
 struct SplitParams {
   const float* q;           // [B][Hq][D]
@@ -86,7 +88,7 @@ struct TileDesc {
   int32_t unit;
   int32_t pidx;  // block index inside this pool
   int32_t p0;    // logical position of the tile's first token
-  int32_t meta;  // valid tokens (0..16) | kFlagPoison | kv head << 16
+  int32_t meta;  // valid tokens (0..16) | kFlagPoison | tile in block << kSubShift | kv head << 16
 };
 
 // ----------------------------------------------------------------------------- small helpers
@@ -283,7 +285,7 @@ struct TileStream {
         }
         const int p0 = j * p.block_size + sub * kTileTokens;
         const int nvalid = min(kTileTokens, L - p0);
-        TileDesc d{unit, pidx, p0, nvalid | (h << 16)};
+        TileDesc d{unit, pidx, p0, nvalid | (sub << kSubShift) | (h << 16)};
         emitted = true;
         ++sub;
         if (sub * kTileTokens >= p.block_size || p0 + kTileTokens >= L) {
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const int nvalid = d.meta & 0xff;
     if (d.unit < 0 || (d.meta & kFlagPoison) || nvalid == 0) return;
     const int h = d.meta >> 16;
-    const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + (d.p0 % p.block_size);
+    const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + ((d.meta >> kSubShift) & kSubMask) * kTileTokens;
     const char* gk = reinterpret_cast<const char*>(p.k_pool + row0 * D) + lane * 16;
     const char* gv = reinterpret_cast<const char*>(p.v_pool + row0 * D) + lane * 16;
     char* sk = ring + static_cast<size_t>(slot) * 2 * TILE + lane * 16;
@@ -645,18 +647,18 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     cp_async_commit();
   }
   int cur_h = 0;
+  int fill = NST - 1, slot = 0;  // ring stage being filled, stage being consumed
 #pragma unroll 1
-  for (int k = 0;; ++k) {
+  for (;;) {
     {
-      const int slot = (k + NST - 1) % NST;
       const TileDesc d = ts.next(p, lane);
-      if (lane == 0) meta[warp][slot] = d;
-      issue(d, slot);
+      if (lane == 0) meta[warp][fill] = d;
+      issue(d, fill);
       cp_async_commit();
+      fill = fill + 1 == NST ? 0 : fill + 1;
     }
     cp_async_wait<NST - 1>();
     __syncwarp();
-    const int slot = k % NST;
     const TileDesc d = meta[warp][slot];
     if (d.unit < 0) break;
     if (d.unit != cur) {
@@ -668,6 +670,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     if (d.meta & kFlagPoison) poisoned = true;
     else if ((d.meta & 0xff) > 0) compute(slot, d);
     __syncwarp();
+    slot = slot + 1 == NST ? 0 : slot + 1;
   }
   if (cur >= 0) finalize(cur, cur_h);
   cp_async_wait<0>();

@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
     const int nvalid = d.meta & 0xff;
     if (d.unit < 0 || (d.meta & kFlagPoison) || nvalid == 0) return;
     const int h = d.meta >> 16;
-    const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + (d.p0 % p.block_size);
+    const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + ((d.meta >> kSubShift) & kSubMask) * kTileTokens;
     const char* gk = reinterpret_cast<const char*>(p.k_pool + row0 * D) + lane * 16;
     const char* gv = reinterpret_cast<const char*>(p.v_pool + row0 * D) + lane * 16;
     char* sk = ring + static_cast<size_t>(slot) * 2 * TILE;
@@ -352,18 +352,18 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
     issue(d, s);
     cp_async_commit();
   }
+  int fill = NST - 1, slot = 0;  // ring stage being filled, stage being consumed
 #pragma unroll 1
-  for (int k = 0;; ++k) {
+  for (;;) {
     {
-      const int slot = (k + NST - 1) % NST;
       const TileDesc d = ts.next(p, lane);
-      if (lane == 0) meta[warp][slot] = d;
-      issue(d, slot);
+      if (lane == 0) meta[warp][fill] = d;
+      issue(d, fill);
       cp_async_commit();
+      fill = fill + 1 == NST ? 0 : fill + 1;
     }
     cp_async_wait<NST - 1>();
     __syncwarp();
-    const int slot = k % NST;
     const TileDesc d = meta[warp][slot];
     if (d.unit < 0) break;
     if (d.unit != cur) {
@@ -375,6 +375,7 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
     if (d.meta & kFlagPoison) poisoned = true;
     else if ((d.meta & 0xff) > 0) compute(slot, d);
     __syncwarp();
+    slot = slot + 1 == NST ? 0 : slot + 1;
   }
   if (cur >= 0) finalize(cur, cur_h);
   cp_async_wait<0>();
