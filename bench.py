@@ -36,6 +36,8 @@ import kvgen  # noqa: E402
 METRIC = "decode-attention µs/step & KV GB/s, fraction of PCIe+HBM roofline"
 HBM_NOMINAL_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 10**6        # B200 L2
+FLUSH_BYTES = 256 << 20       # written between timed steps when the KV of a step fits in L2
 
 
 def parse_args(argv=None):
@@ -114,11 +116,25 @@ class ClockSampler:
                                          stdout=self.file, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
-        time.sleep(0.3)
+            return
+        self._wait_rows(1, 5.0)   # nvidia-smi is up and sampling before the timed region starts
+
+    def _rows(self) -> int:
+        try:
+            with open(self.file.name) as f:
+                return sum(1 for line in f if line.strip())
+        except OSError:
+            return 0
+
+    def _wait_rows(self, n: int, limit_s: float):
+        t0 = time.monotonic()
+        while self._rows() < n and time.monotonic() - t0 < limit_s and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def stop(self) -> dict | None:
         if self.proc is None:
             return None
+        self._wait_rows(self._rows() + 1, 1.0)   # one sample taken at the end of a short timed region
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -305,23 +321,44 @@ def run_dkv(args):
     if attn.status() != 0:
         raise RuntimeError("device status nonzero after warm-up")
 
+    # A step whose KV fits twice in L2 is timed step by step, with a write of
+    # FLUSH_BYTES (larger than L2) between steps and outside their events, so
+    # no step reads KV left in L2 by the previous one.
+    kv_bytes = kv.host_bytes + kv.dev_bytes
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device) if kv_bytes < 2 * L2_BYTES else None
+
+    def timed(fn, steps):
+        if flush_buf is None:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                fn()
+            b.record(stream)
+            b.synchronize()
+            return a.elapsed_time(b) / steps
+        pairs = []
+        for _ in range(steps):
+            flush_buf.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            pairs.append((a, b))
+        pairs[-1][1].synchronize()
+        return sum(a.elapsed_time(b) for a, b in pairs) / steps
+
     # ---- timed region: K steps, device time on the launching stream, per-kernel events inside the library
     clocks = ClockSampler(torch.cuda.current_device())
     barrier()
     torch.cuda.synchronize(device)
     clocks.start()
     dkv.dkv_profile_begin(attn.handle, args.steps)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
+    ms_local = timed(step, args.steps)
     torch.cuda.synchronize(device)
     kernel_ms, kernel_counts = dkv.dkv_profile_end(attn.handle)
     clock_info = clocks.stop()
     barrier()
     launches_per_step = attn.launches()
-    ms_local = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms_local, device)
 
     # ---- end to end through the public API: inputs from pinned host memory, result back to the host
@@ -345,13 +382,7 @@ def run_dkv(args):
             e2e_step()
         torch.cuda.synchronize(device)
         barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        b.record(stream)
-        b.synchronize()
-        e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, device)
+        e2e_ms = max_over_ranks(timed(e2e_step, args.steps), device)
         e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms}
 
@@ -415,7 +446,10 @@ def run_dkv(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
         "config": dict(workload_config(w, world), host_bytes=host_bytes, dev_bytes=dev_bytes, mode=args.mode,
                        query_tokens=tq,
-                       l2="inputs larger than L2: %.0f MiB of KV per step vs 126 MB L2" % ((host_bytes + dev_bytes) / 2**20)),
+                       l2=("inputs larger than L2: %.0f MiB of KV per step vs 126 MB L2" % (kv_bytes / 2**20)
+                           if flush_buf is None else
+                           "L2 flushed between timed steps (%d MiB write outside the step events): %.1f MiB of KV "
+                           "per step vs 126 MB L2" % (FLUSH_BYTES >> 20, kv_bytes / 2**20))),
         "roofline": ({k2: dominant[k2] for k2 in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
                      if dominant else None),
         "roofline_kernels": kernels,

@@ -54,6 +54,7 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kFlagPoison = 1 << 8;
 constexpr int kSubShift = 9;                   // tile index inside its block (block_size <= 1024)
 constexpr int kSubMask = 63;
+constexpr float kLazyMax = 8.f;                // softmax reference max lags the true max by < 2^8
 
 struct SplitParams {
   const float* q;           // [B][Hq][D]
@@ -579,18 +580,33 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       mt[k] = j & 3;
       sc[k] = (tg + 4 * mt[k]) < nvalid ? v[k] : -INFINITY;
     }
-    // ---- online softmax for head gl (max shared by the head's lanes)
+    // ---- online softmax for head gl.  The reference max mrun (shared by the
+    // head's lanes) is raised only when a score of the tile exceeds it by more
+    // than kLazyMax (log2 units), so the weights 2^(s - mrun) stay below
+    // 2^kLazyMax.  The running sum and the output use the same reference, so
+    // the result is exact up to rounding; most tiles skip the cross-lane max,
+    // the rescale factor and the accumulator rescale.
     float tm = sc[0];
 #pragma unroll
     for (int k = 1; k < NH; ++k) tm = fmaxf(tm, sc[k]);
-    tm = head_max(tm);
-    const float mx = fmaxf(mrun, tm);
-    const float alpha = ex2(mrun - mx);
+    if (__any_sync(kFull, tm > mrun + kLazyMax)) {
+      tm = head_max(tm);
+      const float mx = fmaxf(mrun, tm);
+      const float alpha = ex2(mrun - mx);
+      lrun *= alpha;
+      mrun = mx;
+      const float al = __shfl_sync(kFull, alpha, (gT & 3) * HL);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        acc[n][0] *= al;
+        acc[n][1] *= al;
+      }
+    }
     float psum = 0.f;
     float pv[NH];
 #pragma unroll
     for (int k = 0; k < NH; ++k) {
-      pv[k] = ex2(sc[k] - mx);
+      pv[k] = ex2(sc[k] - mrun);
       psum += pv[k];
     }
     if constexpr (G == 4) {
@@ -601,14 +617,12 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       if ((li & 1) == 0) s_p[warp][0][tg][mt[0]] = pv[0];
       if (li & 1) psum = 0.f;  // the odd lane holds a duplicate of its even neighbour's token
     }
-    lrun = lrun * alpha + psum;
-    mrun = mx;
+    lrun += psum;
     __syncwarp();
     // ---- PV on the tensor cores.  A rows 0..7 (lane >> 2): rows 0..3 hi,
     // rows 4..7 lo, of head (lane >> 2) & 3; B = V from the swizzled tile.
     uint32_t a[2] = {0u, 0u};
     const int gA = gT & 3;
-    const float al = __shfl_sync(kFull, alpha, gA * HL);
     if (gA < G) {
       // tokens 2c, 2c+1 (a[0]) and 2c+8, 2c+9 (a[1]); token t lives at [t % 4][t / 4]
       const float* sp = &s_p[warp][gA][0][0];
@@ -620,13 +634,6 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       split_hi_lo<BF16>(pb, hb, lb);
       a[0] = lane < 16 ? ha : la;
       a[1] = lane < 16 ? hb : lb;
-    }
-    if (al != 1.f) {
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        acc[n][0] *= al;
-        acc[n][1] *= al;
-      }
     }
     const int vrow = (lane & 7) | (lane & 8);
 #pragma unroll

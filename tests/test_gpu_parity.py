@@ -229,3 +229,64 @@ def test_staged_prefetch_comparator_matches_zero_copy():
         case.attn.staged(case.q_dev, case.kv, out, None, None)
     assert e.value.code == dkv.DKV_ERR_INVALID_ARG
     case.free()
+
+
+@pytest.mark.parametrize("block_size,d,placement", [
+    (256, 64, "prefix_host"),     # the tiny config with one 256-token block per side
+    (512, 128, "random"),
+    (1024, 128, "random"),        # the largest block: 64 tiles per block
+    (1024, 64, "prefix_host"),
+])
+def test_large_blocks(block_size, d, placement):
+    """Blocks of many tiles: every tile of a block is addressed from its own offset inside the block."""
+    if d == 64 and placement == "prefix_host" and block_size == 256:
+        w = kvgen.TINY_GQA.replace(name="tiny_s256", block_size=256)
+    else:
+        w = kvgen.LLAMA3_8B.replace(name=f"blocks_s{block_size}_d{d}", batch=3, head_dim=d, ctx=(700, 5000),
+                                    block_size=block_size, placement=placement, host_fraction=0.5, seed=block_size + d)
+    case = gc.Case(w)
+    check(case)
+    if w.name == "tiny_s256":
+        assert case.kv.host_split == 1 and case.kv.num_dev_blocks == 1
+    case.free()
+
+
+def test_gqa_equals_mha_with_repeated_kv_heads():
+    """G query heads sharing one KV head give what G copies of that KV head give to one query head each."""
+    w = kvgen.LLAMA3_8B.replace(name="gqa", batch=2, num_q_heads=8, num_kv_heads=2, ctx=(300, 1400), seed=61)
+    gqa = gc.Case(w)
+    a = gqa.run()
+    g = w.num_q_heads // w.num_kv_heads
+    wm = w.replace(name="gqa_as_mha", num_kv_heads=w.num_q_heads)
+    mha = gc.Case.__new__(gc.Case)
+    mha.w, mha.q, mha.lens = wm, gqa.q.copy(), gqa.lens.copy()
+    mha.k, mha.v = np.repeat(gqa.k, g, axis=1), np.repeat(gqa.v, g, axis=1)
+    mha.kv = dkv.PagedKV(mha.k, mha.v, mha.lens, wm.block_size, gc.placement_code(wm), wm.host_fraction, wm.shuffle,
+                         wm.seed)
+    mha.attn = gc.attention_for(wm, max_blocks=max(wm.max_blocks_per_seq(), mha.kv.stride))
+    mha.q_dev = torch.from_numpy(mha.q).cuda()
+    mha.out = torch.empty_like(mha.q_dev)
+    b = mha.run()
+    assert mha.attn.status() == 0
+    assert np.abs(a - b).max() <= 2e-5   # different kernel instances: only fp32 summation order differs
+    assert gc.max_err(a, gqa.oracle()) <= gc.TOL
+    gqa.free()
+    mha.free()
+
+
+def test_output_is_linear_in_v():
+    """V doubled (exact in 16 bits) doubles the output bit for bit: the weights do not depend on V."""
+    w = kvgen.LLAMA3_8B.replace(name="lin_v", batch=2, ctx=(200, 2100), seed=62)
+    case = gc.Case(w)
+    a = case.run()
+    v2 = kvgen.to_bits(kvgen.bits_to_f32(case.v, w.kv_dtype) * 2.0, w.kv_dtype)
+    twice = gc.Case.__new__(gc.Case)
+    twice.w, twice.q, twice.lens, twice.k, twice.v = w, case.q, case.lens, case.k, v2
+    twice.kv = dkv.PagedKV(case.k, v2, case.lens, w.block_size, gc.placement_code(w), w.host_fraction, w.shuffle,
+                           w.seed)
+    twice.attn, twice.q_dev = case.attn, case.q_dev
+    twice.out = torch.empty_like(case.q_dev)
+    b = twice.run()
+    assert np.array_equal(b, 2.0 * a)
+    case.free()
+    twice.free()
