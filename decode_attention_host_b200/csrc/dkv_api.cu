@@ -197,7 +197,10 @@ void plan_splits(const dkv_handle* h, int batch, int stride, int* nsplit, int* b
     *bps = 1;
     return;
   }
-  const long per = static_cast<long>(batch) * num_queries * h->cfg.num_kv_heads;
+  // one unit (b, split, kv head) per warp of a full wave, whatever the number
+  // of query tokens: a unit carries all Tq * G query rows of its kv head
+  (void)num_queries;
+  const long per = static_cast<long>(batch) * h->cfg.num_kv_heads;
   const int target = static_cast<int>((h->units_target + per - 1) / per) > 0
                          ? static_cast<int>((h->units_target + per - 1) / per)
                          : 1;
@@ -290,7 +293,10 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   cudaError_t e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, c.device);
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaDeviceGetAttribute"));
   h->units_target = h->sm_count * 8;  // one unit per warp of a full wave (2 CTAs x 4 warps per SM)
-  h->part_rows = 2ull * G * (static_cast<size_t>(h->units_target) + static_cast<size_t>(c.max_batch) * c.num_kv_heads);
+  // partial rows: batch * Tq * Hq * 2 * nsplit with nsplit <= units_target / (batch * Hkv) + 1 and
+  // Tq * G <= 16 rows per unit (multi-token queries), batch * Tq <= max_batch
+  h->part_rows = 2ull * (static_cast<size_t>(dkv::kMultiMaxRows) * h->units_target +
+                         static_cast<size_t>(G) * c.max_batch * c.num_kv_heads);
   e = cudaFuncSetAttribute(h->host_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(split_smem(c.head_dim, kHostStages)));
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(host kernel)"));

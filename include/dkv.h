@@ -77,7 +77,10 @@ typedef struct CUstream_st* dkv_stream_t; /* the same type as cudaStream_t; NULL
  * dkv_create -- validate cfg and allocate the per-handle workspace on
  * cfg->device: the split-K partial buffers, the device status word, an
  * auxiliary high-priority stream and two events used to fork/join the host
- * and HBM kernels.  On success *out owns all of it until dkv_destroy.
+ * and HBM kernels.  The partial buffers hold 2 * (16 * 8 * SMs + G *
+ * max_batch * Hkv) rows of head_dim + 1 floats (about 20 MB for 148 SMs,
+ * head_dim 128), enough for one split-K unit per warp of a full wave with up
+ * to 16 query rows each.  On success *out owns all of it until dkv_destroy.
  * Errors: INVALID_ARG (null pointers, out-of-range fields), UNSUPPORTED
  * (head_dim or group size), NO_MEMORY, CUDA.
  */
