@@ -442,6 +442,7 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   sp.qscale = h->qscale;
   sp.extra_tokens = nq - 1;
   sp.num_queries = nq;
+  dkv::set_divisors(sp);
   const SplitEntry& host_k = multi ? h->multi_kernel : h->host_kernel;
   const SplitEntry& dev_k = multi ? h->multi_kernel : h->dev_kernel;
   const size_t host_smem = multi ? multi_smem(c.head_dim) : split_smem(c.head_dim, kHostStages);

@@ -56,6 +56,25 @@ constexpr int kSubShift = 9;                   // tile index inside its block (b
 constexpr int kSubMask = 63;
 constexpr float kLazyMax = 8.f;                // softmax reference max lags the true max by < 2^8
 
+// Division by a divisor fixed for the launch, by multiplication (Granlund and
+// Montgomery, "Division by invariant integers using multiplication", 1994):
+// with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1, the quotient
+// n / d equals (umulhi(n, m) + n) >> s for every 0 <= n < 2^31 (the sum then
+// stays below 2^32).  Replaces the per-unit runtime divisions of the kernels.
+struct InvDiv {
+  uint32_t d, m, s;
+  __device__ __forceinline__ int div(int n) const {
+    return static_cast<int>((__umulhi(static_cast<uint32_t>(n), m) + static_cast<uint32_t>(n)) >> s);
+  }
+};
+
+inline InvDiv make_invdiv(int32_t d) {
+  InvDiv r{static_cast<uint32_t>(d), 0u, 0u};
+  while ((1ull << r.s) < static_cast<uint64_t>(d)) ++r.s;
+  r.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << r.s) - static_cast<uint64_t>(d))) / static_cast<uint64_t>(d) + 1);
+  return r;
+}
+
 struct SplitParams {
   const float* q;           // [B][Hq][D]
   const uint16_t* k_pool;   // [nblocks][Hkv][S][D] of this residency
@@ -75,7 +94,15 @@ struct SplitParams {
   float qscale;             // softmax scale * log2(e)
   int32_t extra_tokens;     // tokens past seq_lens that belong to the unit (multi-token queries: Tq - 1)
   int32_t num_queries;      // query tokens per sequence (1 for decode)
+  InvDiv div_hkv, div_nsplit, div_bs;  // hkv, nsplit, block_size (set_divisors)
 };
+
+// Fill the divisor fields from hkv, nsplit and block_size (all >= 1).
+inline void set_divisors(SplitParams& p) {
+  p.div_hkv = make_invdiv(p.hkv);
+  p.div_nsplit = make_invdiv(p.nsplit);
+  p.div_bs = make_invdiv(p.block_size);
+}
 
 struct MergeParams {
   const float* part_o;
@@ -241,14 +268,14 @@ struct TileStream {
   bool started, emitted, bad_len;
 
   __device__ void begin_unit(const SplitParams& p) {
-    h = unit % p.hkv;
-    const int bc = unit / p.hkv;
-    const int c = bc % p.nsplit;
-    b = bc / p.nsplit;
+    const int bc = p.div_hkv.div(unit);
+    h = unit - bc * p.hkv;
+    b = p.div_nsplit.div(bc);
+    const int c = bc - b * p.nsplit;
     L = p.seq_lens[b];
     bad_len = (L < 0 || L + p.extra_tokens > p.max_len);
     L += p.extra_tokens;
-    const int nblk = bad_len ? 0 : (L + p.block_size - 1) / p.block_size;
+    const int nblk = bad_len ? 0 : p.div_bs.div(L + p.block_size - 1);
     j = c * p.bps;
     j_end = min(j + p.bps, nblk);
     sub = 0;
@@ -423,7 +450,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   };
 
   auto init_unit = [&](int unit, int h) {
-    const int b = (unit / p.hkv) / p.nsplit;
+    const int b = p.div_nsplit.div(p.div_hkv.div(unit));
     const int L = p.seq_lens[b];
     float2 C[NP2], S[NP2];
     if constexpr (ROPE) {
@@ -474,9 +501,9 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   };
 
   auto finalize = [&](int unit, int h) {
-    const int bc = unit / p.hkv;
-    const int c = bc % p.nsplit;
-    const int b = bc / p.nsplit;
+    const int bc = p.div_hkv.div(unit);
+    const int b = p.div_nsplit.div(bc);
+    const int c = bc - b * p.nsplit;
     const float ltot = head_sum(lrun);
     // hi rows (lanes 0..15) + lo rows (lanes 16..31) of the same head and columns
 #pragma unroll

@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
   auto freq_of = [&](int i) { return s_freq[i % PPL][i / PPL]; };
 
   auto init_unit = [&](int unit, int h) {
-    const int b = (unit / p.hkv) / p.nsplit;
+    const int b = p.div_nsplit.div(p.div_hkv.div(unit));
     const int L = p.seq_lens[b];
     const int rows[2] = {gT, gT + 8};
     uint32_t hi[2][KS][2], lo[2][KS][2];
@@ -165,9 +165,9 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
   };
 
   auto finalize = [&](int unit, int h) {
-    const int bc = unit / p.hkv;
-    const int c = bc % p.nsplit;
-    const int b = bc / p.nsplit;
+    const int bc = p.div_hkv.div(unit);
+    const int b = p.div_nsplit.div(bc);
+    const int c = bc - b * p.nsplit;
     float t0 = l0, t1 = l1;
     t0 += __shfl_xor_sync(kFull, t0, 1);
     t0 += __shfl_xor_sync(kFull, t0, 2);

@@ -255,6 +255,7 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
   sp.qscale = static_cast<float>(scale * 1.4426950408889634);
   sp.extra_tokens = 0;
   sp.num_queries = 1;
+  dkv::set_divisors(sp);
   const int unit_ctas = (sp.n_units + dkv::kWarps - 1) / dkv::kWarps;
 
   if (host_split > 0) {
