@@ -205,16 +205,25 @@ def recorded_traffic(kernel: str, workload: str):
     return rec
 
 
-def oracle_gbs(w: kvgen.Workload, q, k, v, lens, group_mask) -> tuple[float, float, int]:
-    """Time the fp64 oracle on the (batch, kv head) groups of group_mask: (GB/s, seconds, threads)."""
+CPU_SAMPLE_S = 10.0   # the CPU baseline repeats its sample until at least this much CPU work is timed
+CPU_SAMPLE_MAX_REPS = 200
+
+
+def oracle_gbs(w: kvgen.Workload, q, k, v, lens, group_mask, min_seconds: float = CPU_SAMPLE_S
+               ) -> tuple[float, float, int, int]:
+    """Time the fp64 oracle on the (batch, kv head) groups of group_mask, repeated until about
+    min_seconds have run (once if 0): (GB/s, seconds, threads, repetitions)."""
     import oracle
     dt = oracle.KV_BF16 if w.kv_dtype == kvgen.BF16 else oracle.KV_F16
-    t0 = time.perf_counter()
-    oracle.decode(q, k, v, lens, dt, w.rope_base, group_mask=group_mask)
-    sec = time.perf_counter() - t0
+    reps, sec = 0, 0.0
+    while reps == 0 or (sec < min_seconds and reps < CPU_SAMPLE_MAX_REPS):
+        t0 = time.perf_counter()
+        oracle.decode(q, k, v, lens, dt, w.rope_base, group_mask=group_mask)
+        sec += time.perf_counter() - t0
+        reps += 1
     tokens = sum(int(lens[b]) for b in range(w.batch) for h in range(w.num_kv_heads) if group_mask[b, h])
-    nbytes = tokens * 2 * w.head_dim * 2
-    return nbytes / sec / 1e9, sec, oracle.num_threads()
+    nbytes = tokens * 2 * w.head_dim * 2 * reps
+    return nbytes / sec / 1e9, sec, oracle.num_threads(), reps
 
 
 # ----------------------------------------------------------------------------- reference arm (the oracle)
@@ -237,7 +246,7 @@ def run_reference(args):
         mask = np.zeros((w.batch, w.num_kv_heads), dtype=np.uint8)
         for g in order[(i * per_step) % ngroups:][:per_step]:
             mask.flat[g] = 1
-        gbs, sec, _ = oracle_gbs(w, q, k, v, lens, mask)
+        gbs, sec, _, _ = oracle_gbs(w, q, k, v, lens, mask, min_seconds=0.0)
         if i >= args.warmup:
             times.append(sec)
             nbytes.append(gbs * sec * 1e9)
@@ -434,9 +443,9 @@ def run_dkv(args):
     if keep_logical:
         ngroups = w.batch * w.num_kv_heads
         mask = np.ones((w.batch, w.num_kv_heads), dtype=np.uint8)
-        gbs, sec, threads = oracle_gbs(w, q, k, v, lens, mask)
+        gbs, sec, threads, reps = oracle_gbs(w, q, k, v, lens, mask)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"all {ngroups} (batch, kv head) groups of one step, {sec:.1f} s"}
+               "sample": f"all {ngroups} (batch, kv head) groups of one step, run {reps} times: {sec:.1f} s"}
 
     if e2e is not None:
         e2e["value"] = total / (e2e["ms_per_step"] * 1e-3) / 1e9
