@@ -46,7 +46,7 @@ extern "C" {
 /* ---- return codes ------------------------------------------------------ */
 #define DKV_OK 0
 #define DKV_ERR_INVALID_ARG (-1) /* a pointer, size or enum is out of its documented range */
-#define DKV_ERR_UNSUPPORTED (-2) /* valid request this build does not implement (head dim, group size) */
+#define DKV_ERR_UNSUPPORTED (-2) /* valid request the library does not implement (head dim, group size) */
 #define DKV_ERR_CUDA (-3)        /* a CUDA runtime call failed; see dkv_last_error_string() */
 #define DKV_ERR_NO_MEMORY (-4)   /* device or pinned host allocation failed */
 
