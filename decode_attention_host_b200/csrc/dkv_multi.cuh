@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
   extern __shared__ __align__(128) char smem[];
   __shared__ TileDesc meta[kWarps][NST];
   __shared__ double s_freq[PPL][8];
-  __shared__ float2 s_e[NP2][8], s_f[NP2][8], s_nf[NP2][8];
+  __shared__ float2 s_e[NP2][8], s_f[NP2][8];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -59,7 +59,6 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
     rope_cs(4, w, c, sn);
     reinterpret_cast<float*>(&s_e[r >> 1][l])[r & 1] = c;
     reinterpret_cast<float*>(&s_f[r >> 1][l])[r & 1] = sn;
-    reinterpret_cast<float*>(&s_nf[r >> 1][l])[r & 1] = -sn;
   }
   __syncthreads();
 
@@ -101,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
   int lim0 = 0, lim1 = 0;                      // rows see positions < lim
   bool poisoned = false;
   int cur = -1, cur_h = 0;
-  float2 Cc[NP2], Sc[NP2], NSc[NP2];
+  float2 Cc[NP2], Sc[NP2];
   int next_pos = -1, chain = 0;
 
   auto freq_of = [&](int i) { return s_freq[i % PPL][i / PPL]; };
@@ -196,15 +195,12 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
     const char* sv = sk + TILE;
     const int nvalid = d.meta & 0xff;
     // ---- rotation pass: K tile -> rotated hi (in place) + lo (klo), same swizzled layout
-    float2 C[NP2], S[NP2], NS[NP2];
+    // the rotation state stays in registers while positions continue, with
+    // a fresh fp64-reduced seed at least every 16 tiles (at most 64 fp32 steps)
+    float2 (&C)[NP2] = Cc;
+    float2 (&S)[NP2] = Sc;
     if constexpr (ROPE) {
-      if (d.p0 == next_pos && chain < 4) {
-#pragma unroll
-        for (int j = 0; j < NP2; ++j) {
-          C[j] = Cc[j];
-          S[j] = Sc[j];
-          NS[j] = NSc[j];
-        }
+      if (d.p0 == next_pos && chain < 16) {
         ++chain;
       } else {
 #pragma unroll
@@ -214,7 +210,6 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
           rope_cs(d.p0 + tg, s_freq[2 * j + 1][li], c1, s1);
           C[j] = make_float2(c0, c1);
           S[j] = make_float2(s0, s1);
-          NS[j] = make_float2(-s0, -s1);
         }
         chain = 1;
       }
@@ -233,14 +228,13 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
 #pragma unroll
         for (int j = 0; j < NP2; ++j) {
           const float2 x = X[j], y = Y[j];
-          X[j] = __ffma2_rn(y, NS[j], __fmul2_rn(x, C[j]));
+          const float2 ns = __fmul2_rn(S[j], make_float2(-1.f, -1.f));
+          X[j] = __ffma2_rn(y, ns, __fmul2_rn(x, C[j]));
           Y[j] = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));
-          const float2 e = s_e[j][li], f = s_f[j][li], nf = s_nf[j][li];
-          const float2 cn = __ffma2_rn(NS[j], f, __fmul2_rn(C[j], e));
-          const float2 sn = __ffma2_rn(C[j], f, __fmul2_rn(S[j], e));
-          NS[j] = __ffma2_rn(C[j], nf, __fmul2_rn(NS[j], e));
+          const float2 e = s_e[j][li], f = s_f[j][li];
+          const float2 cn = __ffma2_rn(ns, f, __fmul2_rn(C[j], e));
+          S[j] = __ffma2_rn(C[j], f, __fmul2_rn(S[j], e));
           C[j] = cn;
-          S[j] = sn;
         }
       }
       uint32_t xh[NP2], xl[NP2], yh[NP2], yl[NP2];
@@ -261,15 +255,7 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
         *reinterpret_cast<uint2*>(klo + oy) = make_uint2(yl[0], yl[1]);
       }
     }
-    if constexpr (ROPE) {
-#pragma unroll
-      for (int j = 0; j < NP2; ++j) {
-        Cc[j] = C[j];
-        Sc[j] = S[j];
-        NSc[j] = NS[j];
-      }
-      next_pos = d.p0 + kTileTokens;
-    }
+    if constexpr (ROPE) next_pos = d.p0 + kTileTokens;
     __syncwarp();
     // ---- S = Q K^T on the tensor cores: tokens 0..7 (S0) and 8..15 (S1)
     float S0[4] = {0.f, 0.f, 0.f, 0.f}, S1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -299,25 +285,23 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
       v0[k] = (in && pos < lim0) ? v0[k] : -INFINITY;
       v1[k] = (in && pos < lim1) ? v1[k] : -INFINITY;
     }
+    // The row's reference max (shared by its 4 lanes) is raised only when a
+    // score of the tile exceeds it by more than kLazyMax (log2 units); the
+    // weights 2^(s - m) then stay below 2^kLazyMax and the sum and the output
+    // keep the same reference, so the result is exact up to rounding.
     float tm0 = fmaxf(fmaxf(v0[0], v0[1]), fmaxf(v0[2], v0[3]));
     float tm1 = fmaxf(fmaxf(v1[0], v1[1]), fmaxf(v1[2], v1[3]));
-    tm0 = fmaxf(tm0, __shfl_xor_sync(kFull, tm0, 1));
-    tm0 = fmaxf(tm0, __shfl_xor_sync(kFull, tm0, 2));
-    tm1 = fmaxf(tm1, __shfl_xor_sync(kFull, tm1, 1));
-    tm1 = fmaxf(tm1, __shfl_xor_sync(kFull, tm1, 2));
-    const float mx0 = fmaxf(m0, tm0), mx1 = fmaxf(m1, tm1);
-    const float al0 = ex2(m0 - mx0), al1 = ex2(m1 - mx1);
-    float p0[4], p1[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      p0[k] = ex2(v0[k] - mx0);
-      p1[k] = ex2(v1[k] - mx1);
-    }
-    l0 = l0 * al0 + ((p0[0] + p0[1]) + (p0[2] + p0[3]));
-    l1 = l1 * al1 + ((p1[0] + p1[1]) + (p1[2] + p1[3]));
-    m0 = mx0;
-    m1 = mx1;
-    if (al0 != 1.f || al1 != 1.f) {
+    if (__any_sync(kFull, tm0 > m0 + kLazyMax || tm1 > m1 + kLazyMax)) {
+      tm0 = fmaxf(tm0, __shfl_xor_sync(kFull, tm0, 1));
+      tm0 = fmaxf(tm0, __shfl_xor_sync(kFull, tm0, 2));
+      tm1 = fmaxf(tm1, __shfl_xor_sync(kFull, tm1, 1));
+      tm1 = fmaxf(tm1, __shfl_xor_sync(kFull, tm1, 2));
+      const float mx0 = fmaxf(m0, tm0), mx1 = fmaxf(m1, tm1);
+      const float al0 = ex2(m0 - mx0), al1 = ex2(m1 - mx1);
+      l0 *= al0;
+      l1 *= al1;
+      m0 = mx0;
+      m1 = mx1;
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         acc[n][0] *= al0;
@@ -326,6 +310,14 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
         acc[n][3] *= al1;
       }
     }
+    float p0[4], p1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      p0[k] = ex2(v0[k] - m0);
+      p1[k] = ex2(v1[k] - m1);
+    }
+    l0 += (p0[0] + p0[1]) + (p0[2] + p0[3]);
+    l1 += (p1[0] + p1[1]) + (p1[2] + p1[3]);
     // A fragments of P: {r0 tokens 2c.., r1 tokens 2c.., r0 tokens 8+2c.., r1 tokens 8+2c..}
     uint32_t ph[4], pl[4];
     split_hi_lo<BF16>(make_float2(p0[0], p0[1]), ph[0], pl[0]);
