@@ -206,7 +206,7 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 CPU_SAMPLE_S = 10.0   # the CPU baseline repeats its sample until at least this much CPU work is timed
-CPU_SAMPLE_MAX_REPS = 200
+CPU_SAMPLE_MAX_REPS = 100000
 
 
 def oracle_gbs(w: kvgen.Workload, q, k, v, lens, group_mask, min_seconds: float = CPU_SAMPLE_S
