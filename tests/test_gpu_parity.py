@@ -193,7 +193,8 @@ def _sampled_groups(w, n, seed):
     return mask
 
 
-@pytest.mark.parametrize("name,groups", [("llama3_8b", 6), ("opt_6_7b", 6), ("long_ctx", 2)])
+@pytest.mark.parametrize("name,groups", [("llama3_8b", 6), ("opt_6_7b", 6), ("long_ctx", 2),
+                                         ("sweep_L65536_f0", 3), ("sweep_L262144_f0.5", 2)])
 def test_full_size_sampled_against_oracle(name, groups):
     """Full-size workloads, bench launch configuration; the oracle checks sampled (batch, kv head) groups."""
     w = kvgen.get(name)
