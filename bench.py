@@ -2,12 +2,20 @@
 """Benchmark of zero-copy host/HBM split-KV decode attention on B200.
 
 One step = one dkv_attn_decode call over one batch of the workload: the
-zero-copy host-stream kernel (aux stream), the HBM split-K kernel and the LSE
-merge.  Default workload: the LLaMA-3-8B-shaped layer (B=8, Hq=32, Hkv=8,
-D=128, L=32768, bf16 K/V, 16-token blocks, half the blocks of each sequence
-in mapped pinned host memory, chosen at random).
+pool-lists kernel, the zero-copy host-stream kernel (aux stream), the HBM
+split-K kernel and the LSE merge.  Default workload: the largest single-GPU
+configuration, long-context decode (B=1, Hq=32, Hkv=8, D=128, L=1,048,576
+tokens, bf16 K/V, 64-token blocks, the oldest 90% of blocks in mapped pinned
+host memory and the newest 10% in HBM: 4 GiB of KV per step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dkv|reference]
+                    [--mode zero_copy|staged|planned] [--hbm-budget-frac F]
+
+--mode planned measures the workload at its own placement first, gives the
+host-stream and HBM kernels' measured rates to the offload planner
+(dkv_plan_offload), rebuilds the cache at the planned host fraction and
+reports the planned step: predicted against measured time and the HBM bytes
+the placement frees.
 
 With N > 1 (launched by torchrun) every rank runs an independent replica of
 the workload on its own GPU and PCIe link; rank 0 prints the JSON line with
@@ -45,13 +53,18 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="llama3_8b")
+    ap.add_argument("--workload", default="long_ctx")
     ap.add_argument("--impl", choices=("dkv", "reference"), default="dkv")
-    ap.add_argument("--mode", choices=("zero_copy", "staged"), default="zero_copy",
-                    help="staged: the prefetch comparator (host pool copied into HBM each step)")
+    ap.add_argument("--mode", choices=("zero_copy", "staged", "planned"), default="zero_copy",
+                    help="staged: the prefetch comparator (host pool copied into HBM each step); "
+                         "planned: the placement chosen by the offload planner from measured rates")
+    ap.add_argument("--hbm-budget-frac", type=float, default=-1.0,
+                    help="planned mode: HBM the cache may use, as a fraction of its bytes (< 0: unlimited)")
     ap.add_argument("--queries", type=int, default=1,
                     help="query tokens per sequence (>1: multi-token queries, e.g. speculative verification)")
     ap.add_argument("--host-ctas", type=int, default=0)
+    ap.add_argument("--ctx", type=int, default=0,
+                    help="override the context length (a reduced case of the workload, e.g. for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args(argv)
@@ -88,9 +101,12 @@ def barrier():
         dist.barrier()
 
 
-def workload_for_rank(name: str, rank: int) -> kvgen.Workload:
-    """Replica r draws its own inputs: same shapes and recipe, seed + 1000 r."""
+def workload_for_rank(name: str, rank: int, ctx: int = 0) -> kvgen.Workload:
+    """Replica r draws its own inputs: same shapes and recipe, seed + 1000 r.  ctx > 0 replaces the
+    context length (the workload is then named with a "_ctx<N>" suffix)."""
     w = kvgen.get(name)
+    if ctx > 0:
+        w = w.replace(name=f"{w.name}_ctx{ctx}", ctx=ctx)
     return w if rank == 0 else w.replace(seed=w.seed + 1000 * rank)
 
 
@@ -233,7 +249,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    w = kvgen.get(args.workload)
+    w = workload_for_rank(args.workload, 0, args.ctx)
     lens = kvgen.gen_seq_lens(w)
     q = kvgen.gen_q(w)
     k, v = kvgen.gen_kv(w, lens)
@@ -277,6 +293,88 @@ def workload_config(w: kvgen.Workload, n: int) -> dict:
 
 # ----------------------------------------------------------------------------- our arm
 
+def timed_steps(fn, steps, stream, flush_buf):
+    """Device ms per step of fn over `steps` steps, CUDA events on `stream`.  With flush_buf, each step is
+    timed alone and flush_buf (larger than L2) is written between steps, outside the events."""
+    import torch
+    if flush_buf is None:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / steps
+    pairs = []
+    for _ in range(steps):
+        flush_buf.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        pairs.append((a, b))
+    pairs[-1][1].synchronize()
+    return sum(a.elapsed_time(b) for a, b in pairs) / steps
+
+
+def measure_placement(args, dkv, attn, kv, step, stream, device, b_pcie, hbm_peak, hbm_src, w_name, mode):
+    """Warm-up, the timed region (nothing but the steps and the clock sampler), then a separate
+    attribution pass with the library's per-kernel events.  Returns the measurements of this placement."""
+    import torch
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if attn.status() != 0:
+        raise RuntimeError("device status nonzero after warm-up")
+    kv_bytes = kv.host_bytes + kv.dev_bytes
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device) if kv_bytes < 2 * L2_BYTES else None
+
+    # ---- timed region: K steps, device time on the launching stream
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier()
+    torch.cuda.synchronize(device)
+    clocks.start()
+    ms_local = timed_steps(step, args.steps, stream, flush_buf)
+    torch.cuda.synchronize(device)
+    clock_info = clocks.stop()
+    barrier()
+    launches_per_step = attn.launches()
+    ms = max_over_ranks(ms_local, device)
+
+    # ---- attribution pass (not timed as the step): per-kernel events on each kernel's own stream
+    n_prof = max(1, min(args.steps, 10))
+    dkv.dkv_profile_begin(attn.handle, n_prof)
+    timed_steps(step, n_prof, stream, flush_buf)
+    timeline = dkv.dkv_profile_timeline(attn.handle, n_prof - 1)
+    kernel_ms, kernel_counts = dkv.dkv_profile_end(attn.handle)
+
+    kernels = []
+    host_name = "staged_copy_then_hbm" if mode == "staged" else "host_stream"
+    for idx, name, nbytes, bound, peak, unit_src in (
+            (0, host_name, kv.host_bytes, "pcie", b_pcie, "pinned H2D cudaMemcpyAsync measured in this run"),
+            (1, "hbm_split_k", kv.dev_bytes, "hbm", hbm_peak, hbm_src)):
+        if kernel_counts[idx] == 0:
+            continue
+        avg_ms = kernel_ms[idx] / kernel_counts[idx]
+        achieved = nbytes / (avg_ms * 1e-3) / 1e9
+        traffic = recorded_traffic(name, w_name)
+        kernels.append({"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "peak_source": unit_src, "avg_ms": avg_ms,
+                        "algorithmic_bytes_per_launch": nbytes,
+                        "traffic": traffic.get("bytes_per_launch") if traffic else None,
+                        "traffic_detail": traffic})
+    if kernel_counts[2]:
+        kernels.append({"kernel": "merge", "avg_ms": kernel_ms[2] / kernel_counts[2]})
+    names = ("host_stream", "hbm_split_k", "merge")
+    tl = {n: [timeline[2 * i], timeline[2 * i + 1]] for i, n in enumerate(names) if timeline[2 * i] >= 0}
+    if "host_stream" in tl and "hbm_split_k" in tl:
+        h0, h1 = tl["host_stream"]
+        d0, d1 = tl["hbm_split_k"]
+        tl["overlap_ms"] = max(0.0, min(h1, d1) - max(h0, d0))
+    return {"ms": ms, "clocks": clock_info, "launches_per_step": launches_per_step, "kernels": kernels,
+            "timeline_ms": tl, "flush_buf": flush_buf, "kv_bytes": kv_bytes}
+
+
 def run_dkv(args):
     import torch
     rank, world, local = dist_env()
@@ -285,90 +383,95 @@ def run_dkv(args):
     dist_init("nccl")
     import decode_attention_host_b200 as dkv
 
-    w = workload_for_rank(args.workload, rank)
+    w = workload_for_rank(args.workload, rank, args.ctx)
     q = kvgen.gen_q(w)
     lens = kvgen.gen_seq_lens(w)
     k, v = kvgen.gen_kv(w, lens)
     placement = dkv.DKV_PLACE_PREFIX_HOST if w.placement == "prefix_host" else dkv.DKV_PLACE_RANDOM
     tq = args.queries
-    # multi-token queries: the cache holds L + tq - 1 tokens, query i sits at position L + i
-    kv = dkv.PagedKV(k, v, lens, w.block_size, placement, w.host_fraction, w.shuffle, w.seed, device=local)
-    if tq > 1:
-        kv.seq_lens_dev.copy_(torch.from_numpy(lens - (tq - 1)))
+    planned = args.mode == "planned"
+
+    def paged(f):
+        # multi-token queries: the cache holds L + tq - 1 tokens, query i sits at position L + i
+        c = dkv.PagedKV(k, v, lens, w.block_size, placement, f, w.shuffle, w.seed, device=local)
+        if tq > 1:
+            c.seq_lens_dev.copy_(torch.from_numpy(lens - (tq - 1)))
+        return c
+
+    kv = paged(w.host_fraction)
     attn = dkv.DecodeAttention(w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
                                dkv.DKV_KV_BF16 if w.kv_dtype == kvgen.BF16 else dkv.DKV_KV_F16, w.rope_base,
                                w.batch * tq, kv.stride, device=local, host_ctas=args.host_ctas)
     keep_logical = rank == 0 and world == 1 and not args.no_cpu_baseline and args.queries == 1
-    if not keep_logical:
+    if not keep_logical and not planned:
         del k, v
     q_dev = torch.from_numpy(q).to(device)
     out = torch.empty_like(q_dev)
     stream = torch.cuda.current_stream(device)
     b_pcie = measure_pcie_gbs(device)
+    peaks = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    hbm_src = "MEASURED_PEAKS.json hbm_gbs (copy, measured)" if "hbm_gbs" in peaks else "fallback 6650 GB/s"
 
     if tq > 1:
         q_dev = torch.from_numpy(np.random.default_rng(w.seed).standard_normal(
             (w.batch, tq, w.num_q_heads, w.head_dim)).astype(np.float32)).to(device)
         out = torch.empty_like(q_dev)
+    k_stage = v_stage = None
     if args.mode == "staged":
         blk = w.num_kv_heads * w.block_size * w.head_dim
         k_stage = torch.empty(max(1, kv.host_split * blk), dtype=torch.int16, device=device)
         v_stage = torch.empty_like(k_stage)
 
-        def step():
+    def step():
+        if args.mode == "staged":
             attn.staged(q_dev, kv, out, k_stage, v_stage, stream)
-    elif tq > 1:
-        def step():
+        elif tq > 1:
             attn.multi(q_dev, kv, out, stream)
-    else:
-        def step():
+        else:
             attn(q_dev, kv, out, stream)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(device)
-    if attn.status() != 0:
-        raise RuntimeError("device status nonzero after warm-up")
-
-    # A step whose KV fits twice in L2 is timed step by step, with a write of
-    # FLUSH_BYTES (larger than L2) between steps and outside their events, so
-    # no step reads KV left in L2 by the previous one.
-    kv_bytes = kv.host_bytes + kv.dev_bytes
-    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device) if kv_bytes < 2 * L2_BYTES else None
-
-    def timed(fn, steps):
-        if flush_buf is None:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(steps):
-                fn()
-            b.record(stream)
-            b.synchronize()
-            return a.elapsed_time(b) / steps
-        pairs = []
-        for _ in range(steps):
-            flush_buf.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            pairs.append((a, b))
-        pairs[-1][1].synchronize()
-        return sum(a.elapsed_time(b) for a, b in pairs) / steps
-
-    # ---- timed region: K steps, device time on the launching stream, per-kernel events inside the library
-    clocks = ClockSampler(torch.cuda.current_device())
-    barrier()
-    torch.cuda.synchronize(device)
-    clocks.start()
-    dkv.dkv_profile_begin(attn.handle, args.steps)
-    ms_local = timed(step, args.steps)
-    torch.cuda.synchronize(device)
-    kernel_ms, kernel_counts = dkv.dkv_profile_end(attn.handle)
-    clock_info = clocks.stop()
-    barrier()
-    launches_per_step = attn.launches()
-    ms = max_over_ranks(ms_local, device)
+    meas = measure_placement(args, dkv, attn, kv, step, stream, device, b_pcie, hbm_peak, hbm_src, w.name,
+                             args.mode)
+    planner = None
+    if planned:
+        # The offload planner, fed with the two kernels' rates measured side by side.  Round 0 uses the rates
+        # of the workload's own placement; each later round re-plans from the rates measured at the previous
+        # plan (the rates depend on the operating point), and stops once the fraction settles.
+        def rates_of(m):
+            r = {k["kernel"]: k["achieved"] for k in m["kernels"] if "achieved" in k}
+            return r.get("host_stream", b_pcie * 0.92), r.get("hbm_split_k", hbm_peak)
+        x = float(meas["kv_bytes"])
+        budget = args.hbm_budget_frac * x if args.hbm_budget_frac >= 0 else -1.0
+        host_gbs, hbm_gbs = rates_of(meas)
+        rounds = [{"host_fraction": w.host_fraction, "measured_step_ms": meas["ms"], "host_stream_gbs": host_gbs,
+                   "hbm_split_k_gbs": hbm_gbs}]
+        f_prev = w.host_fraction
+        plan = None
+        for _ in range(2):
+            plan = dkv.dkv_plan_offload(x, host_gbs, hbm_gbs, budget)
+            if abs(plan.host_fraction - f_prev) < 1e-3:
+                break
+            kv.free()
+            kv = paged(plan.host_fraction)
+            meas = measure_placement(args, dkv, attn, kv, step, stream, device, b_pcie, hbm_peak, hbm_src, w.name,
+                                     args.mode)
+            host_gbs, hbm_gbs = rates_of(meas)
+            rounds.append({"host_fraction": plan.host_fraction,
+                           "rates_used_gbs": [rounds[-1]["host_stream_gbs"], rounds[-1]["hbm_split_k_gbs"]],
+                           "predicted_step_ms": plan.step_seconds * 1e3, "measured_step_ms": meas["ms"],
+                           "predicted_over_measured": plan.step_seconds * 1e3 / meas["ms"],
+                           "host_stream_gbs": host_gbs, "hbm_split_k_gbs": hbm_gbs})
+            f_prev = plan.host_fraction
+        last = rounds[-1]
+        planner = {"rounds": rounds, "hbm_budget_bytes": budget if budget >= 0 else None,
+                   "time_optimal_fraction": plan.time_optimal_fraction, "host_fraction": f_prev,
+                   "predicted_step_ms": last.get("predicted_step_ms"), "measured_step_ms": meas["ms"],
+                   "predicted_over_measured": last.get("predicted_over_measured"),
+                   "hbm_bytes_freed": float(kv.host_bytes), "hbm_bytes_used": float(kv.dev_bytes),
+                   "hbm_fraction_freed": kv.host_bytes / max(1, kv.host_bytes + kv.dev_bytes)}
+    ms = meas["ms"]
+    flush_buf = meas["flush_buf"]
 
     # ---- end to end through the public API: inputs from pinned host memory, result back to the host
     e2e = None
@@ -391,7 +494,7 @@ def run_dkv(args):
             e2e_step()
         torch.cuda.synchronize(device)
         barrier()
-        e2e_ms = max_over_ranks(timed(e2e_step, args.steps), device)
+        e2e_ms = max_over_ranks(timed_steps(e2e_step, args.steps, stream, flush_buf), device)
         e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms}
 
@@ -416,26 +519,9 @@ def run_dkv(args):
     host_bytes, dev_bytes = kv.host_bytes, kv.dev_bytes
     total = (host_bytes + dev_bytes) * world
     value = total / (ms * 1e-3) / 1e9
-    peaks = measured_peaks()
-    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
-    hbm_src = "MEASURED_PEAKS.json hbm_gbs (copy, measured)" if "hbm_gbs" in peaks else "fallback 6650 GB/s"
-
-    kernels = []
-    host_name = "staged_copy_then_hbm" if args.mode == "staged" else "host_stream"
-    for idx, name, nbytes, bound, peak, unit_src in (
-            (0, host_name, host_bytes, "pcie", b_pcie, "pinned H2D cudaMemcpyAsync measured in this run"),
-            (1, "hbm_split_k", dev_bytes, "hbm", hbm_peak, hbm_src)):
-        if kernel_counts[idx] == 0:
-            continue
-        avg_ms = kernel_ms[idx] / kernel_counts[idx]
-        achieved = nbytes / (avg_ms * 1e-3) / 1e9
-        traffic = recorded_traffic(name, w.name)
-        kernels.append({"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                        "frac": achieved / peak, "peak_source": unit_src, "avg_ms": avg_ms,
-                        "algorithmic_bytes_per_launch": nbytes,
-                        "traffic": traffic.get("bytes_per_launch") if traffic else None,
-                        "traffic_detail": traffic})
-    dominant = max(kernels, key=lambda r: r["avg_ms"]) if kernels else None
+    kernels = meas["kernels"]
+    bw_kernels = [r for r in kernels if "bound" in r]
+    dominant = max(bw_kernels, key=lambda r: r["avg_ms"]) if bw_kernels else None
     t_star_meas = max(host_bytes / (b_pcie * 1e9), dev_bytes / (hbm_peak * 1e9))
     t_star_nom = max(host_bytes / (b_pcie * 1e9), dev_bytes / (HBM_NOMINAL_GBS * 1e9))
 
@@ -449,11 +535,15 @@ def run_dkv(args):
 
     if e2e is not None:
         e2e["value"] = total / (e2e["ms_per_step"] * 1e-3) / 1e9
+    kv_bytes = meas["kv_bytes"]
+    cfg = workload_config(w, world)
+    if planned:
+        cfg["host_fraction"] = planner["host_fraction"]
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
-        "config": dict(workload_config(w, world), host_bytes=host_bytes, dev_bytes=dev_bytes, mode=args.mode,
+        "config": dict(cfg, host_bytes=host_bytes, dev_bytes=dev_bytes, mode=args.mode,
                        query_tokens=tq,
                        l2=("inputs larger than L2: %.0f MiB of KV per step vs 126 MB L2" % (kv_bytes / 2**20)
                            if flush_buf is None else
@@ -465,12 +555,15 @@ def run_dkv(args):
         "roofline_step": {"t_star_ms_measured_hbm": t_star_meas * 1e3, "frac_measured_hbm": t_star_meas / (ms * 1e-3),
                           "t_star_ms_nominal_hbm": t_star_nom * 1e3, "frac_nominal_hbm": t_star_nom / (ms * 1e-3),
                           "b_pcie_gbs": b_pcie, "b_hbm_measured_gbs": hbm_peak, "b_hbm_nominal_gbs": HBM_NOMINAL_GBS},
+        "kernel_timeline_ms": meas["timeline_ms"],
         "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clock_info,
+        "gpu_launches": meas["launches_per_step"] * args.steps,
+        "clocks": meas["clocks"],
         "cpu_baseline": cpu,
         "parity": parity,
     }
+    if planner is not None:
+        line["planner"] = planner
     print(json.dumps(line), flush=True)
     barrier()
     kv.free()

@@ -31,6 +31,8 @@ DKV_ERR_CUDA = -3
 DKV_ERR_NO_MEMORY = -4
 DKV_STATUS_BAD_BLOCK_ID = 1
 DKV_STATUS_BAD_SEQ_LEN = 2
+DKV_STATUS_COPY_TIMEOUT = 4
+DKV_STATUS_INTERNAL = 8
 DKV_KV_F16 = 0
 DKV_KV_BF16 = 1
 DKV_PLACE_PREFIX_HOST = 0
@@ -40,7 +42,8 @@ EXPORTED = ("dkv_create", "dkv_destroy", "dkv_attn_decode", "dkv_get_status", "d
             "dkv_last_launch_count", "dkv_query_plan", "dkv_host_pool_alloc", "dkv_host_pool_free",
             "dkv_plan_blocks", "dkv_pack_kv", "dkv_profile_begin", "dkv_profile_end",
             "dkv_attn_decode_noalloc", "dkv_plan_offload", "dkv_attn_decode_staged", "dkv_append_kv",
-            "dkv_attn_decode_multi")
+            "dkv_attn_decode_multi", "dkv_debug_rope", "dkv_profile_timeline", "dkv_debug_fail_alloc",
+            "dkv_debug_stall_copy")
 
 
 class DkvConfig(ctypes.Structure):
@@ -96,6 +99,10 @@ def _load() -> ctypes.CDLL:
         "dkv_attn_decode_noalloc": [c.POINTER(DkvConfig), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32,
                                     i32],
         "dkv_profile_end": [vp, c.POINTER(c.c_float), c.POINTER(i32)],
+        "dkv_debug_rope": [i32, i32, c.c_double, vp, vp, i32, vp, vp, vp, i32, vp, vp],
+        "dkv_profile_timeline": [vp, i32, c.POINTER(c.c_float)],
+        "dkv_debug_fail_alloc": [i32],
+        "dkv_debug_stall_copy": [i32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -229,8 +236,33 @@ def dkv_attn_decode_noalloc(cfg: DkvConfig, q, k_host, v_host, k_dev, v_dev, blo
                                        stream, int(batch), int(block_table_stride), int(num_dev_blocks)))
 
 
+def dkv_debug_fail_alloc(nth: int) -> None:
+    """Test only: the nth device allocation of the next dkv_create on this thread fails (0 disarms)."""
+    _check(lib.dkv_debug_fail_alloc(int(nth)))
+
+
+def dkv_debug_stall_copy(enable: bool) -> None:
+    """Test only: the next HBM launch on this thread leaves one tile copy unissued (its wait runs out)."""
+    _check(lib.dkv_debug_stall_copy(1 if enable else 0))
+
+
+def dkv_debug_rope(kv_dtype, head_dim, rope_base, k, tile_pos, num_tiles, k_out, q, q_pos, num_q, q_out,
+                   stream) -> None:
+    """Test only: the decode kernels' RoPE steps on given key tiles and queries."""
+    _check(lib.dkv_debug_rope(int(kv_dtype), int(head_dim), float(rope_base), _p(k), _p(tile_pos), int(num_tiles),
+                              _p(k_out), _p(q), _p(q_pos), int(num_q), _p(q_out), stream))
+
+
 def dkv_profile_begin(h: int, max_calls: int) -> None:
     _check(lib.dkv_profile_begin(h, int(max_calls)))
+
+
+def dkv_profile_timeline(h: int, call: int) -> list[float]:
+    """(start, stop) in ms of the host-stream kernel, the HBM kernel and the merge of one recorded call,
+    from the earliest start; -1 for a kernel that did not run."""
+    t = (ctypes.c_float * 6)()
+    _check(lib.dkv_profile_timeline(h, int(call), t))
+    return list(t)
 
 
 def dkv_profile_end(h: int) -> tuple[list[float], list[int]]:

@@ -16,7 +16,8 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libdkv.so"
 SOURCES = [CSRC / "dkv_api.cu", CSRC / "dkv_noalloc.cu", CSRC / "dkv_host.cpp"]
-HEADERS = [CSRC / "dkv_kernels.cuh", CSRC / "dkv_append.cuh", CSRC / "dkv_multi.cuh", CSRC / "dkv_error.h", ROOT / "include" / "dkv.h"]
+HEADERS = [CSRC / "dkv_kernels.cuh", CSRC / "dkv_append.cuh", CSRC / "dkv_multi.cuh", CSRC / "dkv_error.h",
+           CSRC / "dkv_plan.h", CSRC / "dkv_tma.h", ROOT / "include" / "dkv.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared", "-cudart", "static",

@@ -14,10 +14,14 @@
 #include "dkv_append.cuh"
 #include "dkv_kernels.cuh"
 #include "dkv_multi.cuh"
+#include "dkv_plan.h"
+#include "dkv_tma.h"
 
 namespace {
 
 thread_local std::string g_err;
+thread_local int g_fail_alloc = 0;   // test hook: the n-th device allocation of the next dkv_create fails
+thread_local int g_stall_copy = 0;   // test hook: the next HBM launch leaves one tile copy unissued
 
 int fail(int code, const std::string& msg) {
   g_err = msg;
@@ -53,26 +57,44 @@ struct DeviceGuard {
   }
 };
 
-constexpr int kHostStages = 4;   // ring depth of the zero-copy host kernel (1 CTA per SM, few SMs)
+#ifndef DKV_HOST_STAGES
+#define DKV_HOST_STAGES 4
+#endif
+constexpr int kHostStages = DKV_HOST_STAGES;  // ring depth of the zero-copy host kernel (build-time knob)
 #ifndef DKV_DEV_STAGES
 #define DKV_DEV_STAGES 3
 #endif
 constexpr int kDevStages = DKV_DEV_STAGES;  // ring depth of the HBM kernel (build-time knob)
+#ifndef DKV_DEV_TMA
+#define DKV_DEV_TMA 1
+#endif
+constexpr bool kDevTma = DKV_DEV_TMA != 0;  // HBM kernel tiles by tensor copies (else 16-byte cp.async; build-time knob)
 constexpr int kDefaultHostCtas = 16;
-constexpr int kMinSplitTokens = 64;
+constexpr int kListThreads = 1024;  // threads of the pool-lists kernel
 
-size_t split_smem(int D, int nst) { return static_cast<size_t>(dkv::kWarps) * nst * 2 * dkv::kTileTokens * D * 2; }
+// cudaMalloc, or a simulated out-of-memory failure when the test hook
+// (dkv_debug_fail_alloc) has armed this allocation.
+cudaError_t dev_alloc(void** p, size_t bytes, int* counter) {
+  if (g_fail_alloc > 0 && ++*counter == g_fail_alloc) {
+    g_fail_alloc = 0;
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  return cudaMalloc(p, bytes);
+}
 
-using SplitFn = void (*)(dim3, size_t, cudaStream_t, const dkv::SplitParams&);
+size_t split_smem(int D, int nst) { return dkv::split_smem_bytes(D, nst); }
+
+using SplitFn = void (*)(dim3, size_t, cudaStream_t, const dkv::SplitParams&, const dkv::TileMaps&);
 using SplitKernelPtr = const void*;
 
-template <int D, int G, bool BF16, int NST, bool ROPE>
-void launch_split(dim3 grid, size_t smem, cudaStream_t s, const dkv::SplitParams& p) {
-  dkv::split_kernel<D, G, BF16, NST, ROPE><<<grid, dkv::kThreads, smem, s>>>(p);
+template <int D, int G, bool BF16, int NST, bool ROPE, bool TMA>
+void launch_split(dim3 grid, size_t smem, cudaStream_t s, const dkv::SplitParams& p, const dkv::TileMaps& m) {
+  dkv::split_kernel<D, G, BF16, NST, ROPE, TMA><<<grid, dkv::kThreads, smem, s>>>(p, m);
 }
-template <int D, int G, bool BF16, int NST, bool ROPE>
+template <int D, int G, bool BF16, int NST, bool ROPE, bool TMA>
 const void* split_ptr() {
-  return reinterpret_cast<const void*>(&dkv::split_kernel<D, G, BF16, NST, ROPE>);
+  return reinterpret_cast<const void*>(&dkv::split_kernel<D, G, BF16, NST, ROPE, TMA>);
 }
 
 struct SplitEntry {
@@ -80,12 +102,14 @@ struct SplitEntry {
   SplitKernelPtr ptr;
 };
 
-template <int NST, bool ROPE>
+// TMA: the HBM launch (tiles by tensor copies); otherwise the zero-copy host
+// launch (16-byte cp.async from mapped host memory).
+template <int NST, bool ROPE, bool TMA>
 SplitEntry pick_split_rope(int D, int G, bool bf16) {
-#define DKV_CASE(DD, GG)                                                                                   \
-  if (D == DD && G == GG) {                                                                                \
-    if (bf16) return {&launch_split<DD, GG, true, NST, ROPE>, split_ptr<DD, GG, true, NST, ROPE>()};      \
-    return {&launch_split<DD, GG, false, NST, ROPE>, split_ptr<DD, GG, false, NST, ROPE>()};              \
+#define DKV_CASE(DD, GG)                                                                                     \
+  if (D == DD && G == GG) {                                                                                  \
+    if (bf16) return {&launch_split<DD, GG, true, NST, ROPE, TMA>, split_ptr<DD, GG, true, NST, ROPE, TMA>()}; \
+    return {&launch_split<DD, GG, false, NST, ROPE, TMA>, split_ptr<DD, GG, false, NST, ROPE, TMA>()};         \
   }
   DKV_CASE(64, 1)
   DKV_CASE(64, 2)
@@ -97,13 +121,13 @@ SplitEntry pick_split_rope(int D, int G, bool bf16) {
   return {nullptr, nullptr};
 }
 
-template <int NST>
+template <int NST, bool TMA>
 SplitEntry pick_split(int D, int G, bool bf16, bool rope) {
-  return rope ? pick_split_rope<NST, true>(D, G, bf16) : pick_split_rope<NST, false>(D, G, bf16);
+  return rope ? pick_split_rope<NST, true, TMA>(D, G, bf16) : pick_split_rope<NST, false, TMA>(D, G, bf16);
 }
 
 template <int D, bool BF16, bool ROPE>
-void launch_multi(dim3 grid, size_t smem, cudaStream_t s, const dkv::SplitParams& p) {
+void launch_multi(dim3 grid, size_t smem, cudaStream_t s, const dkv::SplitParams& p, const dkv::TileMaps&) {
   dkv::multi_kernel<D, BF16, ROPE><<<grid, dkv::kThreads, smem, s>>>(p);
 }
 
@@ -120,10 +144,23 @@ SplitEntry pick_multi(int D, bool bf16, bool rope) {
 // shared memory of the multi-token kernel: per warp a 2-stage (K, V) ring and one rotated-K lo tile
 size_t multi_smem(int D) { return static_cast<size_t>(dkv::kWarps) * 5 * dkv::kTileTokens * D * 2; }
 
-using MergeFn = void (*)(dim3, size_t, cudaStream_t, const dkv::MergeParams&);
+// The merge, optionally as a programmatic dependent launch of the split kernel
+// just before it on the stream: its grid is set up while that kernel drains
+// and its first instruction waits for that kernel's results.
+using MergeFn = cudaError_t (*)(dim3, size_t, cudaStream_t, const dkv::MergeParams&, bool);
 template <int D, int NG>
-void launch_merge(dim3 grid, size_t smem, cudaStream_t s, const dkv::MergeParams& p) {
-  dkv::merge_kernel<D, NG><<<grid, NG * D, smem, s>>>(p);
+cudaError_t launch_merge(dim3 grid, size_t smem, cudaStream_t s, const dkv::MergeParams& p, bool dependent) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NG * D);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, dkv::merge_kernel<D, NG>, p);
 }
 
 }  // namespace
@@ -132,18 +169,29 @@ struct dkv_handle {
   dkv_config cfg{};
   int G = 0;
   int sm_count = 0;
-  int units_target = 0;
+  int beside_host = 0;        // HBM-kernel CTAs that fit on an SM beside a host-kernel CTA (0 or 1)
+  int units_target = 0;       // warps of the widest split launch (one resident wave: 2 CTAs per SM)
   size_t part_rows = 0;
   float qscale = 0.f;
   int host_ctas = 0;
   float* part_o = nullptr;
   float* part_lse = nullptr;
   int32_t* status = nullptr;
+  int32_t* work = nullptr;    // [4]: work counters of the host-side and the device-side split launch
+  int2* lists = nullptr;      // [max_batch][max_blocks_per_seq]: per-pool block lists of a mixed call
+  int2* counts = nullptr;     // [max_batch]
   double* inv_freq = nullptr;
   cudaStream_t aux = nullptr;
   cudaEvent_t ev_fork = nullptr;
   cudaEvent_t ev_join = nullptr;
   SplitEntry host_kernel{}, dev_kernel{}, multi_kernel{};
+  // tensor maps of the last device pool and staging pool the HBM kernel read
+  struct PoolMaps {
+    const void* k = nullptr;
+    const void* v = nullptr;
+    long long rows = -1;
+    dkv::TileMaps maps{};
+  } dev_maps, stage_maps;
   MergeFn merge = nullptr;
   const void* ok_host[2] = {nullptr, nullptr};
   const void* ok_dev[4] = {nullptr, nullptr, nullptr, nullptr};
@@ -183,6 +231,9 @@ void release(dkv_handle* h) {
   cudaFree(h->part_o);
   cudaFree(h->part_lse);
   cudaFree(h->status);
+  cudaFree(h->work);
+  cudaFree(h->lists);
+  cudaFree(h->counts);
   cudaFree(h->inv_freq);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   if (h->ev_join) cudaEventDestroy(h->ev_join);
@@ -190,26 +241,46 @@ void release(dkv_handle* h) {
   delete h;
 }
 
-void plan_splits(const dkv_handle* h, int batch, int stride, int* nsplit, int* bps, int num_queries = 1) {
-  const int nblk = stride < h->cfg.max_blocks_per_seq ? stride : h->cfg.max_blocks_per_seq;
-  if (nblk <= 0 || batch <= 0) {
-    *nsplit = 1;
-    *bps = 1;
-    return;
+// Warps a split launch can keep resident: 2 CTAs of kWarps warps per SM, less
+// the SMs' share the zero-copy host kernel holds while it runs beside it.
+long launch_warps(const dkv_handle* h, bool beside_host) {
+  const long ctas = 2L * h->sm_count - (beside_host ? static_cast<long>(h->host_ctas) * (2 - h->beside_host) : 0);
+  return dkv::kWarps * (ctas > 1 ? ctas : 1);
+}
+
+// Whether one CTA of kernel b fits on an SM that holds one CTA of kernel a,
+// by registers and shared memory.
+int fits_beside(const void* a, size_t smem_a, const void* b, size_t smem_b, int device) {
+  cudaFuncAttributes fa{}, fb{};
+  int regs_sm = 0, smem_sm = 0, reserved = 0;
+  if (cudaFuncGetAttributes(&fa, a) != cudaSuccess || cudaFuncGetAttributes(&fb, b) != cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, device) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
   }
-  // one unit (b, split, kv head) per warp of a full wave, whatever the number
-  // of query tokens: a unit carries all Tq * G query rows of its kv head
-  (void)num_queries;
-  const long per = static_cast<long>(batch) * h->cfg.num_kv_heads;
-  const int target = static_cast<int>((h->units_target + per - 1) / per) > 0
-                         ? static_cast<int>((h->units_target + per - 1) / per)
-                         : 1;
-  int min_bps = (kMinSplitTokens + h->cfg.block_size - 1) / h->cfg.block_size;
-  if (min_bps < 1) min_bps = 1;
-  int b = (nblk + target - 1) / target;
-  if (b < min_bps) b = min_bps;
-  *bps = b;
-  *nsplit = (nblk + b - 1) / b;
+  const long regs = static_cast<long>(fa.numRegs + fb.numRegs) * dkv::kThreads;
+  const size_t smem = smem_a + smem_b + fa.sharedSizeBytes + fb.sharedSizeBytes + 2 * static_cast<size_t>(reserved);
+  return regs <= regs_sm && smem <= static_cast<size_t>(smem_sm) ? 1 : 0;
+}
+
+// The tensor maps of a device-resident pool pair of `blocks` blocks (cached per handle).
+int pool_maps(dkv_handle* h, dkv_handle::PoolMaps& cache, const void* k, const void* v, long long blocks,
+              const dkv::TileMaps** out) {
+  const long long rows = blocks * h->cfg.num_kv_heads * h->cfg.block_size;
+  if (rows >= (1LL << 31)) return fail(DKV_ERR_INVALID_ARG, "a pool holds 2^31 or more token rows");
+  if (cache.k != k || cache.v != v || cache.rows != rows) {
+    cache.rows = -1;
+    if (!dkv::encode_pool_map(&cache.maps.k, k, rows, h->cfg.head_dim) ||
+        !dkv::encode_pool_map(&cache.maps.v, v, rows, h->cfg.head_dim))
+      return fail(DKV_ERR_CUDA, "cuTensorMapEncodeTiled rejected the pool's tensor map");
+    cache.k = k;
+    cache.v = v;
+    cache.rows = rows;
+  }
+  *out = &cache.maps;
+  return DKV_OK;
 }
 
 int check_host_pool(dkv_handle* h, const void* p, int which) {
@@ -281,8 +352,8 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   h->qscale = static_cast<float>(scale * 1.4426950408889634);  // * log2(e)
   h->host_ctas = c.host_ctas > 0 ? c.host_ctas : kDefaultHostCtas;
   const bool rope = c.rope_base > 0.0;
-  h->host_kernel = pick_split<kHostStages>(c.head_dim, G, bf16, rope);
-  h->dev_kernel = pick_split<kDevStages>(c.head_dim, G, bf16, rope);
+  h->host_kernel = pick_split<kHostStages, false>(c.head_dim, G, bf16, rope);
+  h->dev_kernel = pick_split<kDevStages, kDevTma>(c.head_dim, G, bf16, rope);
   h->multi_kernel = pick_multi(c.head_dim, bf16, c.rope_base > 0.0);
   h->merge = c.head_dim == 64 ? &launch_merge<64, 16> : &launch_merge<128, 8>;
 
@@ -292,11 +363,15 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   };
   cudaError_t e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, c.device);
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaDeviceGetAttribute"));
-  h->units_target = h->sm_count * 8;  // one unit per warp of a full wave (2 CTAs x 4 warps per SM)
-  // partial rows: batch * Tq * Hq * 2 * nsplit with nsplit <= units_target / (batch * Hkv) + 1 and
-  // Tq * G <= 16 rows per unit (multi-token queries), batch * Tq <= max_batch
+  h->beside_host = fits_beside(h->host_kernel.ptr, split_smem(c.head_dim, kHostStages), h->dev_kernel.ptr,
+                               split_smem(c.head_dim, kDevStages), c.device);
+  h->units_target = static_cast<int>(launch_warps(h, false));
+  // partial rows: batch * Tq * Hq * (host splits + device splits), each launch's
+  // splits <= max(1, units_target / (batch * Hkv)); Tq * G <= 16 rows per unit
+  // (multi-token queries) and batch * Tq <= max_batch
   h->part_rows = 2ull * (static_cast<size_t>(dkv::kMultiMaxRows) * h->units_target +
                          static_cast<size_t>(G) * c.max_batch * c.num_kv_heads);
+  const size_t list_entries = static_cast<size_t>(c.max_batch) * c.max_blocks_per_seq;
   e = cudaFuncSetAttribute(h->host_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(split_smem(c.head_dim, kHostStages)));
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(host kernel)"));
@@ -306,21 +381,27 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   e = cudaFuncSetAttribute(h->multi_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(multi_smem(c.head_dim)));
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(multi-token kernel)"));
-  if (cudaMalloc(&h->part_o, h->part_rows * c.head_dim * sizeof(float)) != cudaSuccess ||
-      cudaMalloc(&h->part_lse, h->part_rows * sizeof(float)) != cudaSuccess ||
-      cudaMalloc(&h->status, sizeof(int32_t)) != cudaSuccess ||
-      cudaMalloc(&h->inv_freq, sizeof(double) * (c.head_dim / 2)) != cudaSuccess) {
+  int nalloc = 0;
+  const bool armed = g_fail_alloc > 0;
+  if (dev_alloc(reinterpret_cast<void**>(&h->part_o), h->part_rows * c.head_dim * sizeof(float), &nalloc) ||
+      dev_alloc(reinterpret_cast<void**>(&h->part_lse), h->part_rows * sizeof(float), &nalloc) ||
+      dev_alloc(reinterpret_cast<void**>(&h->status), sizeof(int32_t), &nalloc) ||
+      dev_alloc(reinterpret_cast<void**>(&h->work), 4 * sizeof(int32_t), &nalloc) ||
+      dev_alloc(reinterpret_cast<void**>(&h->lists), list_entries * sizeof(int2), &nalloc) ||
+      dev_alloc(reinterpret_cast<void**>(&h->counts), c.max_batch * sizeof(int2), &nalloc) ||
+      dev_alloc(reinterpret_cast<void**>(&h->inv_freq), sizeof(double) * (c.head_dim / 2), &nalloc)) {
     cudaGetLastError();
     return bail(fail(DKV_ERR_NO_MEMORY, "workspace allocation failed"));
   }
-  // theta_i(p) = p * base^(-2i/D): the per-pair frequencies, in fp64
+  if (armed) g_fail_alloc = 0;   // the hook covers one dkv_create only
   double freq[64];
-  for (int i = 0; i < c.head_dim / 2; ++i)
-    freq[i] = c.rope_base > 0.0 ? std::pow(c.rope_base, -2.0 * i / static_cast<double>(c.head_dim)) : 0.0;
+  dkv::rope_frequencies(c.rope_base, c.head_dim, freq);
   e = cudaMemcpy(h->inv_freq, freq, sizeof(double) * (c.head_dim / 2), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaMemcpy(inv_freq)"));
   e = cudaMemset(h->status, 0, sizeof(int32_t));
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaMemset(status)"));
+  e = cudaMemset(h->work, 0, 4 * sizeof(int32_t));
+  if (e != cudaSuccess) return bail(cuda_fail(e, "cudaMemset(work counters)"));
   int lo = 0, hi = 0;
   e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaDeviceGetStreamPriorityRange"));
@@ -344,10 +425,11 @@ int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_table_strid
   if (!h || !num_splits || !blocks_per_split) return fail(DKV_ERR_INVALID_ARG, "dkv_query_plan: null argument");
   if (batch < 0 || batch > h->cfg.max_batch || block_table_stride < 1)
     return fail(DKV_ERR_INVALID_ARG, "dkv_query_plan: batch or stride out of range");
-  int ns, b;
-  plan_splits(h, batch, block_table_stride, &ns, &b);
-  *num_splits = ns;
-  *blocks_per_split = b;
+  const int nblk = block_table_stride < h->cfg.max_blocks_per_seq ? block_table_stride : h->cfg.max_blocks_per_seq;
+  const dkv::SplitPlan pl =
+      dkv::plan_split(nblk, static_cast<long>(batch) * h->cfg.num_kv_heads, h->cfg.block_size, launch_warps(h, false), 0);
+  *num_splits = pl.nsplit;
+  *blocks_per_split = pl.bps;
   return DKV_OK;
 }
 
@@ -412,15 +494,30 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   }
 
   const dkv_config& c = h->cfg;
-  int nsplit, bps;
-  plan_splits(h, batch, block_table_stride, &nsplit, &bps, nq);
-  const int nslots = 2 * nsplit;
+  // Launches: the host-side one (zero-copy host kernel on the auxiliary stream,
+  // or for the staged comparator the HBM kernel over the staging pools) and the
+  // device-side one (HBM kernel over the device pool).  With no pool at all the
+  // device-side launch still runs, so that table entries are checked.
+  const bool run_host = host_split > 0;
+  const bool run_dev = num_dev_blocks > 0 || !run_host;
+  const bool concurrent = run_host && !staged;   // host kernel beside the HBM kernel
+  const bool use_lists = run_host && run_dev;    // each launch walks the list of its own pool's blocks
+  const int nblk_cap = block_table_stride < c.max_blocks_per_seq ? block_table_stride : c.max_blocks_per_seq;
+  const long per = static_cast<long>(batch) * c.num_kv_heads;
+  const long host_warps = staged ? launch_warps(h, false) : static_cast<long>(dkv::kWarps) * h->host_ctas;
+  const dkv::SplitPlan ph = dkv::plan_split(nblk_cap, per, c.block_size, host_warps, 0);
+  const dkv::SplitPlan pd = dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, concurrent), 0);
+  const int nsplit_h = run_host ? ph.nsplit : 0;
+  const int nsplit_d = run_dev ? pd.nsplit : 0;
+  const int nslots = nsplit_h + nsplit_d;
   if (static_cast<size_t>(batch) * nq * c.num_q_heads * nslots > h->part_rows)
     return fail(DKV_ERR_INVALID_ARG, "internal: split plan exceeds the workspace");
-  const int n_units = batch * nsplit * c.num_kv_heads;
-  const int nblk_cap = block_table_stride < c.max_blocks_per_seq ? block_table_stride : c.max_blocks_per_seq;
+  const int min_bps = dkv::min_blocks_per_split(c.block_size);
 
   dkv::SplitParams sp{};
+  sp.lists = use_lists ? h->lists : nullptr;
+  sp.counts = h->counts;
+  sp.list_stride = nblk_cap;
   sp.q = q;
   sp.table = block_table;
   sp.seq_lens = seq_lens;
@@ -432,85 +529,121 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   sp.hkv = c.num_kv_heads;
   sp.block_size = c.block_size;
   sp.stride = block_table_stride;
-  sp.nsplit = nsplit;
-  sp.bps = bps;
   sp.nslots = nslots;
   sp.id_total = host_split + num_dev_blocks;
   sp.max_len = nblk_cap * c.block_size;
-  sp.n_units = n_units;
   sp.rope = c.rope_base > 0.0 ? 1 : 0;
   sp.qscale = h->qscale;
   sp.extra_tokens = nq - 1;
   sp.num_queries = nq;
-  dkv::set_divisors(sp);
+  auto launch_params = [&](int nsplit, int bps, int slot_base, bool dev_list, int32_t* work) {
+    dkv::SplitParams lp = sp;
+    lp.nsplit = nsplit;
+    lp.bps = use_lists ? min_bps : bps;
+    lp.slot_base = slot_base;
+    lp.list_dev = dev_list ? 1 : 0;
+    lp.work = work;
+    lp.n_units = batch * nsplit * c.num_kv_heads;
+    dkv::set_divisors(lp);
+    return lp;
+  };
   const SplitEntry& host_k = multi ? h->multi_kernel : h->host_kernel;
   const SplitEntry& dev_k = multi ? h->multi_kernel : h->dev_kernel;
   const size_t host_smem = multi ? multi_smem(c.head_dim) : split_smem(c.head_dim, kHostStages);
   const size_t dev_smem = multi ? multi_smem(c.head_dim) : split_smem(c.head_dim, kDevStages);
+  auto ctas_for = [&](const dkv::SplitParams& lp, int cap) {
+    const int u = (lp.n_units + dkv::kWarps - 1) / dkv::kWarps;
+    return u < cap ? u : cap;
+  };
 
-  const int unit_ctas = (n_units + dkv::kWarps - 1) / dkv::kWarps;
   int launches = 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (host_split > 0 && staged) {
+  static const dkv::TileMaps no_maps{};   // for launches that copy with cp.async
+  if (use_lists) {
+    dkv::ListParams lp{};
+    lp.table = block_table;
+    lp.seq_lens = seq_lens;
+    lp.lists = h->lists;
+    lp.counts = h->counts;
+    lp.stride = block_table_stride;
+    lp.list_stride = nblk_cap;
+    lp.block_size = c.block_size;
+    lp.host_split = host_split;
+    lp.id_total = host_split + num_dev_blocks;
+    lp.max_len = sp.max_len;
+    lp.extra_tokens = nq - 1;
+    lp.invalid_to_dev = 1;
+    dkv::lists_kernel<kListThreads><<<batch, kListThreads, 0, s>>>(lp);
+    DKV_CUDA(cudaGetLastError());
+    ++launches;
+  }
+  bool merge_follows_split = false;   // the merge directly follows a split kernel on `s`
+  if (run_host && staged) {
     // copy engine: pinned host pools -> HBM staging pools, then the HBM kernel reads them
     const size_t bytes = static_cast<size_t>(host_split) * c.num_kv_heads * c.block_size * c.head_dim * 2;
     if ((rc = prof_mark(h, 0, s, false)) != DKV_OK) return rc;
     DKV_CUDA(cudaMemcpyAsync(k_stage, k_host, bytes, cudaMemcpyHostToDevice, s));
     DKV_CUDA(cudaMemcpyAsync(v_stage, v_host, bytes, cudaMemcpyHostToDevice, s));
-    dkv::SplitParams hp = sp;
+    dkv::SplitParams hp = launch_params(nsplit_h, ph.bps, 0, false, h->work);
     hp.k_pool = static_cast<const uint16_t*>(k_stage);
     hp.v_pool = static_cast<const uint16_t*>(v_stage);
     hp.id_lo = 0;
     hp.id_hi = host_split;
-    hp.slot_base = 0;
-    const int dev_ctas = unit_ctas < 2 * h->sm_count ? unit_ctas : 2 * h->sm_count;
-    dev_k.fn(dim3(dev_ctas), dev_smem, s, hp);
+    const dkv::TileMaps* maps = &no_maps;
+    if (!multi && (rc = pool_maps(h, h->stage_maps, k_stage, v_stage, host_split, &maps)) != DKV_OK) return rc;
+    dev_k.fn(dim3(ctas_for(hp, 2 * h->sm_count)), dev_smem, s, hp, *maps);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 0, s, true)) != DKV_OK) return rc;
     ++launches;
-  } else if (host_split > 0) {
+  } else if (run_host) {
     DKV_CUDA(cudaEventRecord(h->ev_fork, s));
     DKV_CUDA(cudaStreamWaitEvent(h->aux, h->ev_fork, 0));
-    dkv::SplitParams hp = sp;
+    dkv::SplitParams hp = launch_params(nsplit_h, ph.bps, 0, false, h->work);
     hp.k_pool = static_cast<const uint16_t*>(k_host);
     hp.v_pool = static_cast<const uint16_t*>(v_host);
     hp.id_lo = 0;
     hp.id_hi = host_split;
-    hp.slot_base = 0;
-    const int grid = unit_ctas < h->host_ctas ? unit_ctas : h->host_ctas;
     if ((rc = prof_mark(h, 0, h->aux, false)) != DKV_OK) return rc;
-    host_k.fn(dim3(grid), host_smem, h->aux, hp);
+    host_k.fn(dim3(ctas_for(hp, h->host_ctas)), host_smem, h->aux, hp, no_maps);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 0, h->aux, true)) != DKV_OK) return rc;
     DKV_CUDA(cudaEventRecord(h->ev_join, h->aux));
     ++launches;
   }
-  if (num_dev_blocks > 0) {
-    dkv::SplitParams dp = sp;
+  if (run_dev) {
+    dkv::SplitParams dp = launch_params(nsplit_d, pd.bps, nsplit_h, true, h->work + 2);
     dp.k_pool = static_cast<const uint16_t*>(k_dev);
     dp.v_pool = static_cast<const uint16_t*>(v_dev);
     dp.id_lo = host_split;
     dp.id_hi = host_split + num_dev_blocks;
-    dp.slot_base = nsplit;
+    if (!multi && g_stall_copy) {
+      dp.stall_first_copy = 1;
+      g_stall_copy = 0;
+    }
+    const dkv::TileMaps* maps = &no_maps;
+    if (!multi && num_dev_blocks > 0 &&
+        (rc = pool_maps(h, h->dev_maps, k_dev, v_dev, num_dev_blocks, &maps)) != DKV_OK)
+      return rc;
     if ((rc = prof_mark(h, 1, s, false)) != DKV_OK) return rc;
-    const int dev_ctas = unit_ctas < 2 * h->sm_count ? unit_ctas : 2 * h->sm_count;  // one resident wave
-    dev_k.fn(dim3(dev_ctas), dev_smem, s, dp);
+    // at most one resident wave of CTAs; units are handed out dynamically, so
+    // CTAs that find no SM free until others finish simply find no work left
+    dev_k.fn(dim3(ctas_for(dp, 2 * h->sm_count)), dev_smem, s, dp, *maps);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 1, s, true)) != DKV_OK) return rc;
     ++launches;
+    merge_follows_split = !concurrent && h->prof_capacity == 0;
   }
-  if (host_split > 0 && !staged) DKV_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
+  if (concurrent) DKV_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
   dkv::MergeParams mp{};
   mp.part_o = h->part_o;
   mp.part_lse = h->part_lse;
   mp.out = out;
   mp.nslots = nslots;
-  mp.nsplit = nsplit;
-  mp.has_host = host_split > 0;
-  mp.has_dev = num_dev_blocks > 0;
+  mp.nsplit = nsplit_h;
+  mp.has_host = run_host;
+  mp.has_dev = run_dev;
   if ((rc = prof_mark(h, 2, s, false)) != DKV_OK) return rc;
-  h->merge(dim3(batch * nq * c.num_q_heads), nslots * sizeof(float), s, mp);
-  DKV_CUDA(cudaGetLastError());
+  DKV_CUDA(h->merge(dim3(batch * nq * c.num_q_heads), nslots * sizeof(float), s, mp, merge_follows_split));
   if ((rc = prof_mark(h, 2, s, true)) != DKV_OK) return rc;
   ++launches;
   h->last_launches = launches;
@@ -628,6 +761,43 @@ int dkv_profile_begin(dkv_handle* h, int32_t max_calls) {
   return DKV_OK;
 }
 
+int dkv_profile_timeline(dkv_handle* h, int32_t call, float* t_ms) {
+  if (!h || !t_ms || call < 0) return fail(DKV_ERR_INVALID_ARG, "dkv_profile_timeline: bad argument");
+  DeviceGuard guard(h->cfg.device);
+  DKV_CUDA(cudaDeviceSynchronize());
+  // the kernels of call `call`: kernel k took part if its call-th event pair was recorded
+  const cudaEvent_t none = nullptr;
+  cudaEvent_t ev[3][2] = {{none, none}, {none, none}, {none, none}};
+  for (int k = 0; k < 3; ++k)
+    if (call < h->prof_used[k]) {
+      ev[k][0] = h->prof_events[k][2 * call];
+      ev[k][1] = h->prof_events[k][2 * call + 1];
+    }
+  // reference: the earliest start among the kernels that ran
+  int ref = -1;
+  for (int k = 0; k < 3 && ref < 0; ++k)
+    if (ev[k][0]) ref = k;
+  if (ref < 0) return fail(DKV_ERR_INVALID_ARG, "dkv_profile_timeline: no kernel of that call was recorded");
+  for (int k = 0; k < 3; ++k) {
+    if (!ev[k][0]) continue;
+    float d = 0.f;
+    DKV_CUDA(cudaEventElapsedTime(&d, ev[ref][0], ev[k][0]));
+    if (d < 0.f) ref = k;
+  }
+  for (int k = 0; k < 3; ++k) {
+    for (int e = 0; e < 2; ++e) {
+      if (!ev[k][0]) {
+        t_ms[2 * k + e] = -1.f;
+        continue;
+      }
+      float d = 0.f;
+      DKV_CUDA(cudaEventElapsedTime(&d, ev[ref][0], ev[k][e]));
+      t_ms[2 * k + e] = d;
+    }
+  }
+  return DKV_OK;
+}
+
 int dkv_profile_end(dkv_handle* h, float* ms, int32_t* counts) {
   if (!h || !ms || !counts) return fail(DKV_ERR_INVALID_ARG, "dkv_profile_end: null argument");
   DeviceGuard guard(h->cfg.device);
@@ -651,6 +821,47 @@ int dkv_profile_end(dkv_handle* h, float* ms, int32_t* counts) {
     counts[k] = h->prof_used[k];
   }
   prof_release(h);
+  return DKV_OK;
+}
+
+int dkv_debug_fail_alloc(int32_t nth) {
+  if (nth < 0) return fail(DKV_ERR_INVALID_ARG, "dkv_debug_fail_alloc: nth must be >= 0");
+  g_fail_alloc = nth;
+  return DKV_OK;
+}
+
+int dkv_debug_stall_copy(int32_t enable) {
+  g_stall_copy = enable ? 1 : 0;
+  return DKV_OK;
+}
+
+int dkv_debug_rope(int32_t kv_dtype, int32_t head_dim, double rope_base, const void* k, const int32_t* tile_pos,
+                   int32_t num_tiles, float* k_out, const float* q, const int32_t* q_pos, int32_t num_q,
+                   float* q_out, dkv_stream_t stream) {
+  if (kv_dtype != DKV_KV_F16 && kv_dtype != DKV_KV_BF16) return fail(DKV_ERR_INVALID_ARG, "dkv_debug_rope: kv_dtype");
+  if (head_dim != 64 && head_dim != 128) return fail(DKV_ERR_UNSUPPORTED, "dkv_debug_rope: head_dim must be 64 or 128");
+  if (!(rope_base > 1.0) || !std::isfinite(rope_base)) return fail(DKV_ERR_INVALID_ARG, "dkv_debug_rope: rope_base must be > 1");
+  if (num_tiles < 0 || num_q < 0 || (num_tiles > 0 && (!k || !tile_pos || !k_out)) ||
+      (num_q > 0 && (!q || !q_pos || !q_out)))
+    return fail(DKV_ERR_INVALID_ARG, "dkv_debug_rope: null pointer or negative count");
+  if ((reinterpret_cast<uintptr_t>(k) & 15u) || (reinterpret_cast<uintptr_t>(k_out) & 7u) ||
+      (reinterpret_cast<uintptr_t>(q) & 7u) || (reinterpret_cast<uintptr_t>(q_out) & 7u))
+    return fail(DKV_ERR_INVALID_ARG, "dkv_debug_rope: k must be 16-byte and k_out, q, q_out 8-byte aligned");
+  if (num_tiles == 0 && num_q == 0) return DKV_OK;
+  dkv::RopeFreqs fr{};
+  dkv::rope_frequencies(rope_base, head_dim, fr.w);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t* k16 = static_cast<const uint16_t*>(k);
+  const bool bf16 = kv_dtype == DKV_KV_BF16;
+  if (head_dim == 64 && bf16)
+    dkv::rope_debug_kernel<64, true><<<1, 32, 0, s>>>(fr, k16, tile_pos, num_tiles, k_out, q, q_pos, num_q, q_out);
+  else if (head_dim == 64)
+    dkv::rope_debug_kernel<64, false><<<1, 32, 0, s>>>(fr, k16, tile_pos, num_tiles, k_out, q, q_pos, num_q, q_out);
+  else if (bf16)
+    dkv::rope_debug_kernel<128, true><<<1, 32, 0, s>>>(fr, k16, tile_pos, num_tiles, k_out, q, q_pos, num_q, q_out);
+  else
+    dkv::rope_debug_kernel<128, false><<<1, 32, 0, s>>>(fr, k16, tile_pos, num_tiles, k_out, q, q_pos, num_q, q_out);
+  DKV_CUDA(cudaGetLastError());
   return DKV_OK;
 }
 

@@ -40,6 +40,7 @@
 // Scores carry scale*log2(e) so the softmax works with exp2.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -55,6 +56,9 @@ constexpr int kFlagPoison = 1 << 8;
 constexpr int kSubShift = 9;                   // tile index inside its block (block_size <= 1024)
 constexpr int kSubMask = 63;
 constexpr float kLazyMax = 8.f;                // softmax reference max lags the true max by < 2^8
+constexpr int kStatusTimeout = 4;              // a tile copy did not complete in time (DKV_STATUS_COPY_TIMEOUT)
+constexpr int kStatusLayout = 8;               // shared memory not aligned for the tile copies (DKV_STATUS_INTERNAL)
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bound of every wait on a tile copy
 
 // Division by a divisor fixed for the launch, by multiplication (Granlund and
 // Montgomery, "Division by invariant integers using multiplication", 1994):
@@ -76,6 +80,11 @@ inline InvDiv make_invdiv(int32_t d) {
 }
 
 struct SplitParams {
+  int32_t* work;            // [2]: next unit to hand out, CTAs finished; zero between launches
+  const int2* lists;        // [B][list_stride]: (logical block, id) of each pool, or nullptr: logical order
+  const int2* counts;       // [B]: (host, device) list lengths
+  int32_t list_stride;
+  int32_t list_dev;         // this launch walks the device list (the back of each row), else the host list
   const float* q;           // [B][Hq][D]
   const uint16_t* k_pool;   // [nblocks][Hkv][S][D] of this residency
   const uint16_t* v_pool;
@@ -85,13 +94,15 @@ struct SplitParams {
   float* part_o;            // [B][Hq][nslots][D]
   float* part_lse;          // [B][Hq][nslots], log2 domain
   int32_t* status;
-  int32_t hq, hkv, block_size, stride, nsplit, bps, nslots, slot_base;
+  int32_t hq, hkv, block_size, stride, nsplit, nslots, slot_base;
+  int32_t bps;              // blocks per split; with lists the minimum, the per-sequence value follows its list
   int32_t id_lo, id_hi;     // ids in [id_lo, id_hi) live in this pool at (id - id_lo)
   int32_t id_total;         // ids in [0, id_total) are valid in some pool
   int32_t max_len;          // largest valid seq_len
   int32_t n_units;          // B * nsplit * Hkv
   int32_t rope;             // 0: no rotation
   float qscale;             // softmax scale * log2(e)
+  int32_t stall_first_copy; // test hook: warp 0 of CTA 0 arms its first tile's barrier but issues no copy
   int32_t extra_tokens;     // tokens past seq_lens that belong to the unit (multi-token queries: Tq - 1)
   int32_t num_queries;      // query tokens per sequence (1 for decode)
   InvDiv div_hkv, div_nsplit, div_bs;  // hkv, nsplit, block_size (set_divisors)
@@ -108,7 +119,19 @@ struct MergeParams {
   const float* part_o;
   const float* part_lse;
   float* out;               // [B][Hq][D]
-  int32_t nslots, nsplit, has_host, has_dev;
+  int32_t nslots;           // slots per row: host splits, then device splits
+  int32_t nsplit;           // host slots (the first nsplit of each row)
+  int32_t has_host, has_dev;
+};
+
+// The per-pool block lists of one call with blocks in both pools.
+struct ListParams {
+  const int32_t* table;     // [B][stride]
+  const int32_t* seq_lens;  // [B]
+  int2* lists;              // [B][list_stride]
+  int2* counts;             // [B]
+  int32_t stride, list_stride, block_size, host_split, id_total, max_len, extra_tokens;
+  int32_t invalid_to_dev;   // ids outside both pools go to the device list (else to the host list)
 };
 
 // One tile of the copy stream.  unit < 0 marks the end of the stream.
@@ -136,12 +159,171 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// ---- tile copies by the tensor memory accelerator (HBM launch)
+//
+// A K or V tile (16 token rows of D 16-bit elements) arrives as D/64 boxes of
+// 16 rows x 64 elements (128 bytes per row) with the 128-byte swizzle: inside
+// each 1024-byte group of 8 rows, 16-byte chunk c of row r lands at chunk
+// c ^ (r mod 8).  tile_off gives that layout for every producer (the tensor
+// copies of the HBM launch, the 16-byte cp.async of the host launch) and
+// every consumer (the score and PV loops), so 8 lanes that read one row, and
+// the 8 rows of one ldmatrix phase, each touch 8 distinct bank groups.
+
+// Tensor maps of the K and V pools of one launch (unused by cp.async launches).
+struct TileMaps {
+  CUtensorMap k, v;
+};
+
+// Byte offset of 16-byte chunk `chunk` (0 .. D/8-1) of token row `row` in a tile.
+__device__ __forceinline__ int tile_off(int row, int chunk) {
+  return (chunk >> 3) * (kTileTokens * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for phase `parity` of the barrier, giving up after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (unsigned i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+// Orders this thread's earlier generic-proxy accesses to shared memory before
+// its later async-proxy (tensor copy) writes to it.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// One box of the tensor map at (x, y) into shared memory, completing on `bar`
+// (CTA-local destination; no multicast).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
 // cos/sin of pos * w with the angle reduced modulo 2*pi in fp64 first.
 __device__ __forceinline__ void rope_cs(int pos, double w, float& c, float& s) {
   const double th = static_cast<double>(pos) * w;
   const double n = rint(th * 0.15915494309189535);        // 1 / (2*pi)
   const double r = fma(-n, 6.283185307179586, th);        // |r| <= pi (+ rounding)
   __sincosf(static_cast<float>(r), &s, &c);
+}
+
+// ----------------------------------------------------------------------------- RoPE of the split kernel
+//
+// Lane li of a token group owns the NeoX pairs i = li*PPL + r, r < PPL, held
+// as NP2 = PPL/2 float2 values: element j of a row's "X" array holds dims
+// (li*PPL + 2j, li*PPL + 2j + 1), the "Y" array the same dims + D/2.  The
+// tables below are filled once per CTA; the decode kernels and dkv_debug_rope
+// run the same functions on them.
+
+constexpr int kRopeChainTiles = 16;  // tiles that may follow one fp64-reduced seed
+
+template <int PPL>
+struct RopeTables {
+  double freq[PPL][8];                 // [r][li]: base^(-2i/D), i = li*PPL + r
+  float2 e[PPL / 2][8], f[PPL / 2][8]; // cos / sin of the 4-position step, pairs (2j, 2j+1)
+};
+
+// Fill the tables from the D/2 frequencies (all threads of the block; the
+// caller synchronises).  rope == false stores zero frequencies.
+template <int D>
+__device__ __forceinline__ void rope_fill_tables(RopeTables<D / 16>& t, const double* inv_freq, bool rope,
+                                                 int tid, int nthreads) {
+  constexpr int PPL = D / 16;
+  for (int i = tid; i < D / 2; i += nthreads) {
+    const double w = rope ? inv_freq[i] : 0.0;
+    const int l = i / PPL, r = i % PPL;
+    t.freq[r][l] = w;
+    float c, sn;
+    rope_cs(4, w, c, sn);
+    reinterpret_cast<float*>(&t.e[r >> 1][l])[r & 1] = c;
+    reinterpret_cast<float*>(&t.f[r >> 1][l])[r & 1] = sn;
+  }
+}
+
+// cos / sin of position pos for the pairs of lane li.
+template <int PPL>
+__device__ __forceinline__ void rope_seed(const RopeTables<PPL>& t, int li, int pos, float2 (&C)[PPL / 2],
+                                          float2 (&S)[PPL / 2]) {
+#pragma unroll
+  for (int j = 0; j < PPL / 2; ++j) {
+    float c0, s0, c1, s1;
+    rope_cs(pos, t.freq[2 * j][li], c0, s0);
+    rope_cs(pos, t.freq[2 * j + 1][li], c1, s1);
+    C[j] = make_float2(c0, c1);
+    S[j] = make_float2(s0, s1);
+  }
+}
+
+// Start of a K tile whose first token (of this lane's token group tg) sits at
+// p0 + tg: continue the rotation state when the tile follows the previous
+// one (p0 == next_pos) and fewer than kRopeChainTiles tiles have shared the
+// current seed, else take a fresh fp64-reduced seed.
+template <int PPL>
+__device__ __forceinline__ void rope_tile_start(const RopeTables<PPL>& t, int li, int tg, int p0, int& next_pos,
+                                                int& chain, float2 (&C)[PPL / 2], float2 (&S)[PPL / 2]) {
+  if (p0 == next_pos && chain < kRopeChainTiles) {
+    ++chain;
+  } else {
+    rope_seed<PPL>(t, li, p0 + tg, C, S);
+    chain = 1;
+  }
+  next_pos = p0 + 16;
+}
+
+// Rotate one key row by the angle state (C, S): x' = x c - y s, y' = y c + x s;
+// then advance the state 4 positions with the step factors (E, F).  After the
+// fourth row of a tile the state is that of the tile 16 positions on.
+template <int NP2>
+__device__ __forceinline__ void rope_rotate_advance(float2 (&X)[NP2], float2 (&Y)[NP2], float2 (&C)[NP2],
+                                                    float2 (&S)[NP2], const float2 (&E)[NP2],
+                                                    const float2 (&F)[NP2]) {
+#pragma unroll
+  for (int j = 0; j < NP2; ++j) {
+    const float2 x = X[j], y = Y[j];
+    const float2 ns = __fmul2_rn(S[j], make_float2(-1.f, -1.f));
+    X[j] = __ffma2_rn(y, ns, __fmul2_rn(x, C[j]));      // x c - y s
+    Y[j] = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));    // y c + x s
+    // (C + iS)(E + iF)
+    const float2 cn = __ffma2_rn(ns, F[j], __fmul2_rn(C[j], E[j]));
+    S[j] = __ffma2_rn(C[j], F[j], __fmul2_rn(S[j], E[j]));
+    C[j] = cn;
+  }
+}
+
+// A query pair (x = dims i, y = dims i + D/2) rotated by (C, S) and scaled by qs.
+__device__ __forceinline__ void rope_query(float2 x, float2 y, float2 C, float2 S, float2 qs, float2& X, float2& Y) {
+  const float2 xr = __fmul2_rn(x, C);
+  const float2 yr = __fmul2_rn(y, C);
+  const float2 ys = __fmul2_rn(y, S);
+  X = __fmul2_rn(make_float2(xr.x - ys.x, xr.y - ys.y), qs);   // x c - y s
+  Y = __fmul2_rn(__ffma2_rn(x, S, yr), qs);                    // y c + x s
 }
 
 // Two consecutive 16-bit elements (one 32-bit word) widened to an fp32 pair.
@@ -260,12 +442,29 @@ __device__ __forceinline__ void split_hi_lo(float2 p, uint32_t& hi, uint32_t& lo
 // ----------------------------------------------------------------------------- tile stream
 
 // Enumerates, for one warp, the tiles of this residency over its units.  All
-// lanes run it in lockstep with identical results; block-table reads are
-// uniform (one broadcast load per block).
+// lanes run it in lockstep with identical results; block-table and list reads
+// are uniform (one broadcast load per block).  Units are handed out one at a
+// time from the launch's work counter, so a warp that finishes early takes
+// the next unit and CTAs that start late find the work already taken.
+//
+// Without lists, split c of sequence b covers the logical blocks
+// [c*bps, (c+1)*bps) and skips those of the other pool.  With lists (a call
+// whose blocks sit in both pools), split c covers entries
+// [c*n', (c+1)*n') of the sequence's list of this pool's blocks, n' =
+// max(bps, ceil(n/nsplit)), so every split of a launch holds blocks of its
+// own pool and the work of a launch is even whatever the placement.
 struct TileStream {
-  int unit, unit_stride;
-  int b, h, L, j, j_end, sub, pidx;
+  int unit;
+  int b, h, L, j, j_end, sub, pidx, blk;
+  const int2* lbase;
   bool started, emitted, bad_len;
+
+  __device__ void grab(const SplitParams& p, int lane) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(p.work, 1);
+    unit = __shfl_sync(kFull, u, 0);
+    started = false;
+  }
 
   __device__ void begin_unit(const SplitParams& p) {
     const int bc = p.div_hkv.div(unit);
@@ -275,16 +474,21 @@ struct TileStream {
     L = p.seq_lens[b];
     bad_len = (L < 0 || L + p.extra_tokens > p.max_len);
     L += p.extra_tokens;
-    const int nblk = bad_len ? 0 : p.div_bs.div(L + p.block_size - 1);
-    j = c * p.bps;
-    j_end = min(j + p.bps, nblk);
+    if (p.lists) {
+      const int2 cnt = p.counts[b];
+      const int n = bad_len ? 0 : (p.list_dev ? cnt.y : cnt.x);
+      lbase = p.lists + static_cast<size_t>(b) * p.list_stride + (p.list_dev ? p.list_stride - n : 0);
+      const int per = max(p.bps, p.div_nsplit.div(n + p.nsplit - 1));
+      j = c * per;
+      j_end = min(j + per, n);
+    } else {
+      const int nblk = bad_len ? 0 : p.div_bs.div(L + p.block_size - 1);
+      j = c * p.bps;
+      j_end = min(j + p.bps, nblk);
+    }
     sub = 0;
     emitted = false;
     started = true;
-  }
-  __device__ void next_unit() {
-    unit += unit_stride;
-    started = false;
   }
 
   __device__ TileDesc next(const SplitParams& p, int lane) {
@@ -293,12 +497,20 @@ struct TileStream {
       if (bad_len) {
         if (lane == 0) atomicOr(p.status, 2);
         TileDesc d{unit, 0, 0, kFlagPoison | (h << 16)};
-        next_unit();
+        grab(p, lane);
         return d;
       }
       while (j < j_end) {
         if (sub == 0) {
-          const int id = p.table[static_cast<size_t>(b) * p.stride + j];
+          int id;
+          if (p.lists) {
+            const int2 e = lbase[j];
+            blk = e.x;
+            id = e.y;
+          } else {
+            blk = j;
+            id = p.table[static_cast<size_t>(b) * p.stride + j];
+          }
           if (id >= p.id_lo && id < p.id_hi) {
             pidx = id - p.id_lo;
           } else if (id >= 0 && id < p.id_total) {
@@ -311,7 +523,7 @@ struct TileStream {
             return TileDesc{unit, 0, 0, kFlagPoison | (h << 16)};
           }
         }
-        const int p0 = j * p.block_size + sub * kTileTokens;
+        const int p0 = blk * p.block_size + sub * kTileTokens;
         const int nvalid = min(kTileTokens, L - p0);
         TileDesc d{unit, pidx, p0, nvalid | (sub << kSubShift) | (h << 16)};
         emitted = true;
@@ -324,18 +536,124 @@ struct TileStream {
       }
       const bool was_emitted = emitted;
       const int u = unit;
-      next_unit();
+      grab(p, lane);
       if (!was_emitted) return TileDesc{u, 0, 0, h << 16};  // empty unit: still reported once
     }
     return TileDesc{-1, 0, 0, 0};
   }
 };
 
+// End of a split launch: lets a dependent launch (the merge) be scheduled,
+// then the last CTA to finish clears the work counter for the next launch on
+// the same workspace.  Every warp of every CTA has stopped taking units by
+// the time the last CTA counts itself.
+__device__ __forceinline__ void finish_launch(int32_t* work) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned done = atomicAdd(reinterpret_cast<unsigned*>(work + 1), 1u);
+    if (done == gridDim.x - 1) {
+      atomicExch(work, 0);
+      atomicExch(work + 1, 0);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------- pool lists
+
+// One CTA per sequence: the blocks j < ceil((L_b + extra)/S) of its table row,
+// split by pool into (logical block, id) entries kept in logical order; host
+// blocks fill the front of the row, device blocks its back.  A sequence with
+// an invalid length gets empty lists (the split kernels poison its units).
+// The row is read in coalesced chunks of T entries: a first pass counts the
+// device entries (where the device list starts), a second places every entry
+// at its rank, from warp ballots and the warps' totals in shared memory.
+template <int T>
+__global__ void __launch_bounds__(T) lists_kernel(const ListParams p) {
+  static_assert(T % 32 == 0 && T <= 1024, "block of whole warps");
+  constexpr int NW = T / 32;
+  __shared__ int2 s_warp[NW];
+  __shared__ int s_red[NW];
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int L0 = p.seq_lens[b];
+  const long long Le = static_cast<long long>(L0) + p.extra_tokens;
+  const int n = (L0 < 0 || Le > p.max_len) ? 0 : static_cast<int>((Le + p.block_size - 1) / p.block_size);
+  const int32_t* row = p.table + static_cast<size_t>(b) * p.stride;
+  auto to_dev = [&](int id) {
+    const bool valid = id >= 0 && id < p.id_total;
+    return valid ? id >= p.host_split : p.invalid_to_dev != 0;
+  };
+  // pass 1: device entries of the row
+  int nd = 0;
+  for (int j = tid; j < n; j += T) nd += to_dev(row[j]) ? 1 : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nd += __shfl_xor_sync(kFull, nd, o);
+  if (lane == 0) s_red[warp] = nd;
+  __syncthreads();
+  int td = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) td += s_red[w];
+  // pass 2: ranks, chunk by chunk
+  int2* out = p.lists + static_cast<size_t>(b) * p.list_stride;
+  const unsigned lt = (1u << lane) - 1u;
+  int base_h = 0, base_d = p.list_stride - td;
+  for (int c0 = 0; c0 < n; c0 += T) {
+    const int j = c0 + tid;
+    const bool live = j < n;
+    const int id = live ? row[j] : 0;
+    const bool dev = live && to_dev(id);
+    const bool host = live && !dev;
+    const unsigned bh = __ballot_sync(kFull, host);
+    const unsigned bd = __ballot_sync(kFull, dev);
+    if (lane == 0) s_warp[warp] = make_int2(__popc(bh), __popc(bd));
+    __syncthreads();
+    int oh = 0, od = 0, ch = 0, cd = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const int2 v = s_warp[w];
+      if (w < warp) {
+        oh += v.x;
+        od += v.y;
+      }
+      ch += v.x;
+      cd += v.y;
+    }
+    if (host) out[base_h + oh + __popc(bh & lt)] = make_int2(j, id);
+    if (dev) out[base_d + od + __popc(bd & lt)] = make_int2(j, id);
+    base_h += ch;
+    base_d += cd;
+    __syncthreads();   // s_warp is rewritten by the next chunk
+  }
+  if (tid == 0) p.counts[b] = make_int2(base_h, td);
+}
+
 // ----------------------------------------------------------------------------- split kernel
 
-template <int D, int G, bool BF16, int NST, bool ROPE>
-__global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
+// Shared memory of the split kernel besides the tile rings (all of it is
+// dynamic, rings first, so the rings start at the 1024-byte aligned base of
+// the block's shared memory).
+template <int PPL, int NST>
+struct SplitSmemTail {
+  uint64_t bar[kWarps][NST];                 // per ring stage: completion of its tensor copies
+  TileDesc meta[kWarps][NST];
+  alignas(16) float s_p[kWarps][4][4][4];    // softmax weights of the tile: [head][token group][m]
+  RopeTables<PPL> rope;
+};
+
+// Dynamic shared memory of split_kernel<D, *, *, NST, *, *>.
+__host__ __device__ constexpr size_t split_smem_bytes(int D, int nst) {
+  return static_cast<size_t>(kWarps) * nst * 2 * kTileTokens * D * 2 +
+         (D == 64 ? sizeof(SplitSmemTail<4, 4>) : sizeof(SplitSmemTail<8, 4>));
+}
+
+template <int D, int G, bool BF16, int NST, bool ROPE, bool TMA>
+__global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p, const __grid_constant__ TileMaps maps) {
   static_assert(G >= 1 && G <= 4, "query group of 1, 2 or 4 heads");
+  static_assert(NST <= 4, "SplitSmemTail is sized for up to 4 stages");
   constexpr int PPL = D / 16;                  // NeoX pairs per lane
   constexpr int NP2 = PPL / 2;                 // fp32 pairs per half-row per lane
   constexpr int ROW = D * 2;                   // bytes of one token row
@@ -343,11 +661,13 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   constexpr int CPR = ROW / 16;                // 16-byte chunks per row
   constexpr int NT = D / 8;                    // 8-wide output column tiles of the PV mma
   static_assert(G <= 4, "hi rows 0..3 and lo rows 4..7 of the PV mma");
-  extern __shared__ __align__(128) char smem[];
-  __shared__ TileDesc meta[kWarps][NST];
-  __shared__ double s_freq[PPL][8];            // [r][li]: base^(-2i/D), i = li*PPL + r
-  __shared__ float2 s_e[NP2][8], s_f[NP2][8];  // 4-token step: cos, sin (pairs)
-  __shared__ __align__(16) float s_p[kWarps][4][4][4];  // softmax weights of the tile: [head][token group][m]
+  extern __shared__ __align__(1024) char split_smem[];
+  char* const smem = split_smem;
+  SplitSmemTail<PPL, NST>& tail =
+      *reinterpret_cast<SplitSmemTail<PPL, NST>*>(smem + static_cast<size_t>(kWarps) * NST * 2 * TILE);
+  auto& meta = tail.meta;
+  auto& s_rope = tail.rope;
+  auto& s_p = tail.s_p;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -357,66 +677,120 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   const int cT = lane & 3;                     // column pair of the mma fragments
   char* ring = smem + static_cast<size_t>(warp) * NST * 2 * TILE;
 
-  for (int i = threadIdx.x; i < D / 2; i += kThreads) {
-    const double w = ROPE ? p.inv_freq[i] : 0.0;
-    const int l = i / PPL, r = i % PPL;
-    s_freq[r][l] = w;
-    float c, sn;
-    rope_cs(4, w, c, sn);
-    float* e = reinterpret_cast<float*>(&s_e[r >> 1][l]) + (r & 1);
-    float* f = reinterpret_cast<float*>(&s_f[r >> 1][l]) + (r & 1);
-    *e = c;
-    *f = sn;
+  if constexpr (TMA) {
+    // the swizzled tensor copies need 1024-byte aligned tiles; report and do
+    // nothing rather than copy into a misaligned ring
+    if (smem_u32(smem) & 1023u) {
+      if (threadIdx.x == 0) atomicOr(p.status, kStatusLayout);
+      finish_launch(p.work);
+      return;
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int s = 0; s < NST; ++s) mbar_init(smem_u32(&tail.bar[warp][s]), 1);
+      mbar_init_fence();
+    }
   }
+  rope_fill_tables<D>(s_rope, p.inv_freq, ROPE, threadIdx.x, kThreads);
   __syncthreads();
 
   // 4-position step factors of this lane's pairs, kept in registers
   float2 re[NP2], rf[NP2];
 #pragma unroll
   for (int j = 0; j < NP2; ++j) {
-    re[j] = s_e[j][li];
-    rf[j] = s_f[j][li];
+    re[j] = s_rope.e[j][li];
+    rf[j] = s_rope.f[j][li];
   }
 
   TileStream ts;
-  ts.unit = blockIdx.x * kWarps + warp;
-  ts.unit_stride = gridDim.x * kWarps;
-  ts.started = false;
+  ts.grab(p, lane);
 
-  // Copy chunk e = lane + 32 k of a tile: K rows are stored as they come; V rows
-  // have their 16-byte chunks XOR-swizzled by (row mod 8) so that ldmatrix,
-  // which reads one chunk column of 8 rows, touches 8 distinct bank groups.
-  // For ROW = 256 the swizzled offsets repeat every 4 copies (plus 2 KB).
+  // Tile copies.  TMA: lane 0 arms the stage's barrier with the tile's bytes
+  // and issues D/64 boxes for K and for V; a stage with nothing to copy gets a
+  // plain arrival, so every stage completes exactly once per use.  cp.async:
+  // copy e = lane + 32 k moves 16-byte chunk (e mod CPR) of row (e / CPR);
+  // its shared-memory offset repeats every 4 copies plus 1024 bytes (8 rows).
   constexpr int KCOPIES = kTileTokens * CPR / 32;
-  int vofs[4];
+  int dofs[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int e = lane + 32 * k;
-    vofs[k] = swz<ROW>(e / CPR, e % CPR);
+    dofs[k] = tile_off(e / CPR, e % CPR);
   }
+  uint32_t phase = 0;     // per stage: parity of its next completion (TMA)
+  uint32_t inflight = 0;  // per stage: tensor copies issued and not yet waited for (TMA)
+  bool broken = false;    // a copy did not complete in time: no more copies, every later tile poisoned (TMA)
   auto issue = [&](const TileDesc& d, int slot) {
     const int nvalid = d.meta & 0xff;
-    if (d.unit < 0 || (d.meta & kFlagPoison) || nvalid == 0) return;
+    const bool copy = !(d.unit < 0 || (d.meta & kFlagPoison) || nvalid == 0);
     const int h = d.meta >> 16;
-    const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + ((d.meta >> kSubShift) & kSubMask) * kTileTokens;
-    const char* gk = reinterpret_cast<const char*>(p.k_pool + row0 * D) + lane * 16;
-    const char* gv = reinterpret_cast<const char*>(p.v_pool + row0 * D) + lane * 16;
-    char* sk = ring + static_cast<size_t>(slot) * 2 * TILE + lane * 16;
-    char* sv = ring + static_cast<size_t>(slot) * 2 * TILE + TILE;
-    if (nvalid == kTileTokens) {
+    const int sub = (d.meta >> kSubShift) & kSubMask;
+    char* sk = ring + static_cast<size_t>(slot) * 2 * TILE;
+    char* sv = sk + TILE;
+    if constexpr (TMA) {
+      if (broken) return;
+      if (lane == 0) {
+        const uint32_t bar = smem_u32(&tail.bar[warp][slot]);
+        if (copy) {
+          const int row0 = (d.pidx * p.hkv + h) * p.block_size + sub * kTileTokens;
+          fence_proxy_async();
+          mbar_arrive_expect_tx(bar, 2 * TILE);
+          // the test hook leaves this one stage armed with nothing to complete it
+          const bool stall = p.stall_first_copy && blockIdx.x == 0 && warp == 0 && inflight == 0 && phase == 0;
+          if (!stall) {
 #pragma unroll
-      for (int k = 0; k < KCOPIES; ++k) {
-        cp_async16(sk + 512 * k, gk + 512 * k, 16);
-        cp_async16(sv + vofs[k & 3] + (k >> 2) * 2048, gv + 512 * k, 16);
+            for (int x = 0; x < D / 64; ++x) {
+              tma_load_2d(smem_u32(sk + x * kTileTokens * 128), &maps.k, 64 * x, row0, bar);
+              tma_load_2d(smem_u32(sv + x * kTileTokens * 128), &maps.v, 64 * x, row0, bar);
+            }
+          }
+        } else {
+          mbar_arrive(bar);
+        }
       }
+      if (copy) inflight |= 1u << slot;
     } else {
+      if (!copy) return;
+      const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + sub * kTileTokens;
+      const char* gk = reinterpret_cast<const char*>(p.k_pool + row0 * D) + lane * 16;
+      const char* gv = reinterpret_cast<const char*>(p.v_pool + row0 * D) + lane * 16;
 #pragma unroll
       for (int k = 0; k < KCOPIES; ++k) {
-        const int r = (lane + 32 * k) / CPR;
-        const int nb = r < nvalid ? 16 : 0;
-        cp_async16(sk + 512 * k, nb ? gk + 512 * k : gk - lane * 16, nb);
-        cp_async16(sv + vofs[k & 3] + (k >> 2) * 2048, nb ? gv + 512 * k : gv - lane * 16, nb);
+        const int o = dofs[k & 3] + (k >> 2) * 1024;
+        const int nb = (nvalid == kTileTokens || (lane + 32 * k) / CPR < nvalid) ? 16 : 0;
+        cp_async16(sk + o, nb ? gk + 512 * k : gk - lane * 16, nb);
+        cp_async16(sv + o, nb ? gv + 512 * k : gv - lane * 16, nb);
       }
+    }
+  };
+  // Completion of stage `slot` before its tile is read.  TMA: bounded wait on
+  // the stage's barrier; rows of V past the sequence end hold whatever the
+  // block stores there, so they are zeroed (their weights are 0, but 0 * NaN
+  // is not).  Returns false if the tile cannot be used.
+  auto await_stage = [&](const TileDesc& d, int slot) {
+    if constexpr (TMA) {
+      if (broken) return false;
+      const bool ok = mbar_wait_bounded(smem_u32(&tail.bar[warp][slot]), (phase >> slot) & 1u);
+      if (!__all_sync(kFull, ok)) {
+        broken = true;
+        if (lane == 0) atomicOr(p.status, kStatusTimeout);
+        return false;
+      }
+      phase ^= 1u << slot;
+      inflight &= ~(1u << slot);
+      const int nvalid = d.meta & 0xff;
+      if (d.unit >= 0 && !(d.meta & kFlagPoison) && nvalid > 0 && nvalid < kTileTokens) {
+        char* sv = ring + static_cast<size_t>(slot) * 2 * TILE + TILE;
+        for (int e = lane; e < (kTileTokens - nvalid) * CPR; e += 32)
+          *reinterpret_cast<uint4*>(sv + tile_off(nvalid + e / CPR, e % CPR)) = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async();   // before a later tensor copy overwrites this stage
+      }
+      __syncwarp();
+      return true;
+    } else {
+      cp_async_wait<NST - 1>();
+      __syncwarp();
+      return true;
     }
   };
 
@@ -438,23 +812,12 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   float2 Cc[NP2], Sc[NP2];
   int next_pos = -1, chain = 0;
 
-  auto seeds = [&](int pos, float2 (&C)[NP2], float2 (&S)[NP2]) {
-#pragma unroll
-    for (int j = 0; j < NP2; ++j) {
-      float c0, s0, c1, s1;
-      rope_cs(pos, s_freq[2 * j][li], c0, s0);
-      rope_cs(pos, s_freq[2 * j + 1][li], c1, s1);
-      C[j] = make_float2(c0, c1);
-      S[j] = make_float2(s0, s1);
-    }
-  };
-
   auto init_unit = [&](int unit, int h) {
     const int b = p.div_nsplit.div(p.div_hkv.div(unit));
     const int L = p.seq_lens[b];
     float2 C[NP2], S[NP2];
     if constexpr (ROPE) {
-      seeds(L, C, S);
+      rope_seed<PPL>(s_rope, li, L, C, S);
     } else {
 #pragma unroll
       for (int j = 0; j < NP2; ++j) {
@@ -470,11 +833,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       for (int j = 0; j < NP2; ++j) {
         const float2 x = *reinterpret_cast<const float2*>(qg + li * PPL + 2 * j);
         const float2 y = *reinterpret_cast<const float2*>(qg + D / 2 + li * PPL + 2 * j);
-        const float2 xr = __fmul2_rn(x, C[j]);
-        const float2 yr = __fmul2_rn(y, C[j]);
-        const float2 ys = __fmul2_rn(y, S[j]);
-        QX[g][j] = __fmul2_rn(make_float2(xr.x - ys.x, xr.y - ys.y), qs);   // x c - y s
-        QY[g][j] = __fmul2_rn(__ffma2_rn(x, S[j], yr), qs);                  // y c + x s
+        rope_query(x, y, C[j], S[j], qs, QX[g][j], QY[g][j]);
       }
     }
     mrun = -1e30f;
@@ -533,14 +892,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     // ---- scores: rotate K rows on the fly (CUDA cores, fp32 pairs).  The
     // rotation state (Cc, Sc) carries over when this tile continues the
     // previous one; a fresh fp64-reduced seed at least every 16 tiles.
-    if constexpr (ROPE) {
-      if (d.p0 == next_pos && chain < 16) {
-        ++chain;
-      } else {
-        seeds(d.p0 + tg, Cc, Sc);
-        chain = 1;
-      }
-    }
+    if constexpr (ROPE) rope_tile_start<PPL>(s_rope, li, tg, d.p0, next_pos, chain, Cc, Sc);
     float2 (&C)[NP2] = Cc;
     float2 (&S)[NP2] = Sc;
     float v[4 * G];  // partial scores, index g * 4 + m
@@ -548,23 +900,11 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     for (int m = 0; m < 4; ++m) {
       const int t = tg + 4 * m;
       float2 X[NP2], Y[NP2];
-      const char* krow = sk + t * ROW + li * PPL * 2;
-      load_pairs<NP2, BF16>(krow, X);
-      load_pairs<NP2, BF16>(krow + D, Y);
-      if constexpr (ROPE) {
-#pragma unroll
-        for (int j = 0; j < NP2; ++j) {
-          const float2 x = X[j], y = Y[j];
-          const float2 ns = __fmul2_rn(S[j], make_float2(-1.f, -1.f));
-          X[j] = __ffma2_rn(y, ns, __fmul2_rn(x, C[j]));      // x c - y s
-          Y[j] = __ffma2_rn(x, S[j], __fmul2_rn(y, C[j]));    // y c + x s
-          // advance 4 positions: (C + iS)(E + iF); after m = 3 this is the
-          // first token of the tile 16 positions on
-          const float2 cn = __ffma2_rn(ns, rf[j], __fmul2_rn(C[j], re[j]));
-          S[j] = __ffma2_rn(C[j], rf[j], __fmul2_rn(S[j], re[j]));
-          C[j] = cn;
-        }
-      }
+      constexpr int XB = 0, YB = D;            // byte offsets of the row's two halves
+      const int xb = XB + li * PPL * 2, yb = YB + li * PPL * 2;
+      load_pairs<NP2, BF16>(sk + tile_off(t, xb >> 4) + (xb & 15), X);
+      load_pairs<NP2, BF16>(sk + tile_off(t, yb >> 4) + (yb & 15), Y);
+      if constexpr (ROPE) rope_rotate_advance<NP2>(X, Y, C, S, re, rf);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float2 a = __ffma2_rn(QY[g][0], Y[0], __fmul2_rn(QX[g][0], X[0]));
@@ -576,7 +916,6 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
         v[g * 4 + m] = a.x + a.y;
       }
     }
-    if constexpr (ROPE) next_pos = d.p0 + kTileTokens;
     // ---- reduce-scatter over the 8 lanes of the token group: halve the value
     // set at each xor step; lane li ends with scores g*4+m = li*(4G/8) + k
     constexpr int NV = 4 * G;
@@ -666,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
 #pragma unroll
     for (int qd = 0; qd < D / 16; ++qd) {
       uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(sv + swz<ROW>(vrow, 2 * qd + (lane >> 4)), b0, b1, b2, b3);
+      ldsm_x4_t(sv + tile_off(vrow, 2 * qd + (lane >> 4)), b0, b1, b2, b3);
       mma16816_top<BF16>(acc[2 * qd], a, b0, b1);
       mma16816_top<BF16>(acc[2 * qd + 1], a, b2, b3);
     }
@@ -678,7 +1017,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const TileDesc d = ts.next(p, lane);
     if (lane == 0) meta[warp][s] = d;
     issue(d, s);
-    cp_async_commit();
+    if constexpr (!TMA) cp_async_commit();
   }
   int cur_h = 0;
   int fill = NST - 1, slot = 0;  // ring stage being filled, stage being consumed
@@ -688,12 +1027,12 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       const TileDesc d = ts.next(p, lane);
       if (lane == 0) meta[warp][fill] = d;
       issue(d, fill);
-      cp_async_commit();
+      if constexpr (!TMA) cp_async_commit();
       fill = fill + 1 == NST ? 0 : fill + 1;
     }
-    cp_async_wait<NST - 1>();
     __syncwarp();
     const TileDesc d = meta[warp][slot];
+    const bool usable = await_stage(d, slot);
     if (d.unit < 0) break;
     if (d.unit != cur) {
       if (cur >= 0) finalize(cur, cur_h);
@@ -701,13 +1040,93 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       cur_h = d.meta >> 16;
       init_unit(cur, cur_h);
     }
-    if (d.meta & kFlagPoison) poisoned = true;
+    if ((d.meta & kFlagPoison) || !usable) poisoned = true;
     else if ((d.meta & 0xff) > 0) compute(slot, d);
     __syncwarp();
     slot = slot + 1 == NST ? 0 : slot + 1;
   }
   if (cur >= 0) finalize(cur, cur_h);
-  cp_async_wait<0>();
+  if constexpr (TMA) {
+    // after a timed-out copy, give the copies still in flight a bounded time to
+    // land before the block's shared memory is released
+    if (inflight) {
+#pragma unroll 1
+      for (int s = 0; s < NST; ++s)
+        if (inflight & (1u << s)) mbar_wait_bounded(smem_u32(&tail.bar[warp][s]), (phase >> s) & 1u);
+    }
+  } else {
+    cp_async_wait<0>();
+  }
+  finish_launch(p.work);
+}
+
+// ----------------------------------------------------------------------------- RoPE check kernel
+
+// The D/2 RoPE frequencies passed by value (head_dim <= 128).
+struct RopeFreqs {
+  double w[64];
+};
+
+// dkv_debug_rope: one warp runs the split kernel's RoPE steps on its own data.
+// Key tiles are walked in order, as a warp walks the tiles of its units: the
+// same lane layout, seeds, 4-position recurrence and chaining rule, so row r
+// of tile i is rotated at position tile_pos[i] + r exactly as the decode
+// kernel rotates a K row it holds in shared memory.  Queries are rotated as
+// init_unit rotates them, with a scale of 1.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(32) rope_debug_kernel(const __grid_constant__ RopeFreqs fr, const uint16_t* k,
+                                                        const int32_t* tile_pos, int num_tiles, float* k_out,
+                                                        const float* q, const int32_t* q_pos, int num_q,
+                                                        float* q_out) {
+  constexpr int PPL = D / 16;
+  constexpr int NP2 = PPL / 2;
+  __shared__ RopeTables<PPL> t;
+  const int lane = threadIdx.x;
+  const int tg = lane >> 3;
+  const int li = lane & 7;
+  rope_fill_tables<D>(t, fr.w, true, lane, 32);
+  __syncthreads();
+  float2 E[NP2], F[NP2], C[NP2], S[NP2];
+#pragma unroll
+  for (int j = 0; j < NP2; ++j) {
+    E[j] = t.e[j][li];
+    F[j] = t.f[j][li];
+  }
+  int next_pos = -1, chain = 0;
+  for (int i = 0; i < num_tiles; ++i) {
+    rope_tile_start<PPL>(t, li, tg, tile_pos[i], next_pos, chain, C, S);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const size_t row = static_cast<size_t>(i) * kTileTokens + tg + 4 * m;
+      const char* src = reinterpret_cast<const char*>(k + row * D) + li * PPL * 2;
+      float2 X[NP2], Y[NP2];
+      load_pairs<NP2, BF16>(src, X);
+      load_pairs<NP2, BF16>(src + D, Y);
+      rope_rotate_advance<NP2>(X, Y, C, S, E, F);
+      float* o = k_out + row * D + li * PPL;
+#pragma unroll
+      for (int j = 0; j < NP2; ++j) {
+        *reinterpret_cast<float2*>(o + 2 * j) = X[j];
+        *reinterpret_cast<float2*>(o + D / 2 + 2 * j) = Y[j];
+      }
+    }
+  }
+  for (int n = 0; n < num_q; ++n) {
+    float2 Cq[NP2], Sq[NP2];
+    rope_seed<PPL>(t, li, q_pos[n], Cq, Sq);
+    const float* qn = q + static_cast<size_t>(n) * D + li * PPL;
+    float* o = q_out + static_cast<size_t>(n) * D + li * PPL;
+#pragma unroll
+    for (int j = 0; j < NP2; ++j) {
+      float2 X, Y;
+      rope_query(*reinterpret_cast<const float2*>(qn + 2 * j), *reinterpret_cast<const float2*>(qn + D / 2 + 2 * j),
+                 Cq[j], Sq[j], make_float2(1.f, 1.f), X, Y);
+      if (tg == 0) {
+        *reinterpret_cast<float2*>(o + 2 * j) = X;
+        *reinterpret_cast<float2*>(o + D / 2 + 2 * j) = Y;
+      }
+    }
+  }
 }
 
 // ----------------------------------------------------------------------------- merge kernel
@@ -719,6 +1138,9 @@ __global__ void __launch_bounds__(NG * D) merge_kernel(const MergeParams p) {
   __shared__ float red_m[NG * D / 32], red_z[NG * D / 32];
   __shared__ int red_nan[NG * D / 32];
   __shared__ float part[NG][D];
+  // launched as a programmatic dependent of the split kernel: wait until that
+  // grid has completed and its partials are visible (no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   const float* lse = p.part_lse + static_cast<size_t>(row) * p.nslots;

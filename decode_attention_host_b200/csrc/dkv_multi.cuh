@@ -63,9 +63,7 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
   __syncthreads();
 
   TileStream ts;
-  ts.unit = blockIdx.x * kWarps + warp;
-  ts.unit_stride = gridDim.x * kWarps;
-  ts.started = false;
+  ts.grab(p, lane);
 
   constexpr int KCOPIES = kTileTokens * CPR / 32;
   int vofs[4];
@@ -371,6 +369,7 @@ __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
   }
   if (cur >= 0) finalize(cur, cur_h);
   cp_async_wait<0>();
+  finish_launch(p.work);
 }
 
 }  // namespace dkv

@@ -53,6 +53,9 @@ extern "C" {
 /* ---- device-side status bits (read with dkv_get_status) ----------------- */
 #define DKV_STATUS_BAD_BLOCK_ID 1 /* a block table entry is outside both pools */
 #define DKV_STATUS_BAD_SEQ_LEN 2  /* seq_lens[b] < 0 or beyond the table / handle capacity */
+#define DKV_STATUS_COPY_TIMEOUT 4 /* a tile copy into shared memory did not complete within 2 s; the
+                                     affected rows are NaN (the kernel stopped copying and returned) */
+#define DKV_STATUS_INTERNAL 8     /* the HBM kernel found its shared memory misaligned and did nothing */
 
 typedef enum { DKV_KV_F16 = 0, DKV_KV_BF16 = 1 } dkv_kv_dtype;
 
@@ -75,12 +78,14 @@ typedef struct CUstream_st* dkv_stream_t; /* the same type as cudaStream_t; NULL
 
 /*
  * dkv_create -- validate cfg and allocate the per-handle workspace on
- * cfg->device: the split-K partial buffers, the device status word, an
- * auxiliary high-priority stream and two events used to fork/join the host
- * and HBM kernels.  The partial buffers hold 2 * (16 * 8 * SMs + G *
- * max_batch * Hkv) rows of head_dim + 1 floats (about 20 MB for 148 SMs,
- * head_dim 128), enough for one split-K unit per warp of a full wave with up
- * to 16 query rows each.  On success *out owns all of it until dkv_destroy.
+ * cfg->device: the split-K partial buffers, the device status word, two work
+ * counters per split launch, the per-pool block lists, an auxiliary
+ * high-priority stream and two events used to fork/join the host and HBM
+ * kernels.  The partial buffers hold 2 * (16 * 8 * SMs + G * max_batch * Hkv)
+ * rows of head_dim + 1 floats (about 20 MB for 148 SMs, head_dim 128), enough
+ * for one split-K unit per warp of a full wave with up to 16 query rows each;
+ * the block lists take 8 * max_batch * max_blocks_per_seq bytes.  On success
+ * *out owns all of it until dkv_destroy.
  * Errors: INVALID_ARG (null pointers, out-of-range fields), UNSUPPORTED
  * (head_dim or group size), NO_MEMORY, CUDA.
  */
@@ -197,11 +202,18 @@ DKV_API int dkv_get_status(dkv_handle* h, int32_t* status);
 DKV_API const char* dkv_last_error_string(void);
 
 /* dkv_last_launch_count -- number of kernels the handle's last successful
- * dkv_attn_decode launched (host stream, HBM split-K, merge). */
+ * dkv_attn_decode launched: with blocks in both pools the pool-lists kernel,
+ * the zero-copy host kernel, the HBM split-K kernel and the merge (4); with
+ * one pool, that pool's split kernel and the merge (2). */
 DKV_API int dkv_last_launch_count(const dkv_handle* h, int32_t* count);
 
-/* dkv_query_plan -- the split-K decomposition dkv_attn_decode would use for
- * (batch, block_table_stride): splits per sequence and blocks per split. */
+/* dkv_query_plan -- the split-K decomposition of the HBM kernel of a
+ * dkv_attn_decode call whose blocks all sit in HBM, for (batch,
+ * block_table_stride): splits per sequence and blocks per split.  The splits
+ * never make more units (batch * splits * Hkv) than the kernel's resident
+ * warps.  With host blocks as well, each launch splits the list of its own
+ * pool's blocks of every sequence, and the HBM launch plans for the warps
+ * left beside the zero-copy host kernel. */
 DKV_API int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_table_stride, int32_t* num_splits,
                    int32_t* blocks_per_split);
 
@@ -215,23 +227,29 @@ DKV_API int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_tab
  *
  * dkv_attn_decode_noalloc -- the same computation as dkv_attn_decode, with
  * the configuration passed per call and no handle.  It allocates nothing:
- * its scratch (status word, RoPE frequencies, split partials) is one fixed
- * array of DKV_NOALLOC_SCRATCH_BYTES compiled into the library, held on every
- * GPU that loads the library until the process exits.
+ * its scratch (status word, work counters, RoPE frequencies, per-pool block
+ * lists, split partials) is one fixed array of DKV_NOALLOC_SCRATCH_BYTES
+ * compiled into the library, held on every GPU that loads the library until
+ * the process exits.
  *   cfg          read for this call only; cfg->max_batch is ignored, the
  *                other fields mean what they mean for dkv_create.
  *   status_out   device int32 or NULL: receives the DKV_STATUS_* bits of
  *                this call (the scratch status word is cleared at its start).
  *   other arguments as for dkv_attn_decode.  All kernels run in order on
- *   `stream` (the host-stream and HBM kernels do not overlap here).
+ *   `stream` (the host-stream and HBM kernels do not overlap here): a small
+ *   set-up kernel (frequencies, cleared status and counters), with blocks in
+ *   both pools the pool-lists kernel, the split kernel of each pool and the
+ *   merge -- one launch more than dkv_attn_decode.
  * The first call on a device looks up the device address of the scratch
  * array (cudaGetSymbolAddress) and sets the kernels' shared-memory limits;
  * make that first call before any stream capture.  Every call on a device
  * shares the one array and finds the previous call's contents in it, so calls
  * that may overlap on the GPU (other streams, other threads) race: order them.
- * A batch whose partials cannot fit (batch * num_q_heads beyond about
- * DKV_NOALLOC_SCRATCH_BYTES / (8 * (head_dim + 1))) is rejected with
- * DKV_ERR_INVALID_ARG before anything is launched.  No cudaMalloc, cudaFree
+ * The number of splits is cut down until the partials fit; a batch for which
+ * even one split per pool in use cannot fit (batch * num_q_heads beyond about
+ * DKV_NOALLOC_SCRATCH_BYTES / (4 * (head_dim + 1) * pools in use), less 8
+ * bytes per table block of every sequence when both pools hold blocks) is
+ * rejected with DKV_ERR_INVALID_ARG before anything is launched.  No cudaMalloc, cudaFree
  * or other allocating call is made. */
 #define DKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const float* q, const void* k_host, const void* v_host,
@@ -240,6 +258,46 @@ DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const float* q, const
                                     dkv_stream_t stream, int32_t batch, int32_t block_table_stride,
                                     int32_t num_dev_blocks);
 
+/* ---- allocation-failure injection (test only) ----------------------------
+ * dkv_debug_fail_alloc -- TEST ONLY: makes the nth device allocation (1-based)
+ * of the next dkv_create on the calling thread fail as if the GPU were out of
+ * memory; 0 disarms.  The hook is cleared by the first dkv_create that
+ * reaches its allocations, whether or not it failed.  Lets tests check that
+ * a failed create returns DKV_ERR_NO_MEMORY, frees what it had allocated and
+ * leaves the device usable, without exhausting real GPU memory.  dkv_create
+ * makes 7 device allocations.  Errors: INVALID_ARG (nth < 0). */
+DKV_API int dkv_debug_fail_alloc(int32_t nth);
+
+/* dkv_debug_stall_copy -- TEST ONLY: in the next dkv_attn_decode on the
+ * calling thread that launches the HBM kernel, warp 0 of its first CTA arms
+ * the barrier of its first tile copy but issues no copy, so its bounded wait
+ * runs out (about 2 s): the call must then report DKV_STATUS_COPY_TIMEOUT,
+ * write NaN for that warp's units and leave the device usable.  The hook is
+ * cleared by that call; 0 disarms it.  Always returns DKV_OK. */
+DKV_API int dkv_debug_stall_copy(int32_t enable);
+
+/* ---- RoPE check (test only) ----------------------------------------------
+ * dkv_debug_rope -- TEST ONLY: applies NeoX RoPE exactly as the decode
+ * kernels do, so that the rotation can be compared element by element with an
+ * exact reference at large positions (DirectKV README, opening summary: the
+ * attention kernel applies "Neox RoPE rotation" to the keys it loads).  One
+ * warp walks the key tiles in order, as a decode warp walks the tiles of its
+ * units: the same lane layout, fp64-reduced seed angles, 4-position fp32
+ * recurrence and chaining rule (a tile that starts 16 positions after the
+ * previous one continues the rotation state; at most 16 tiles share one
+ * seed).  Queries are rotated by the decode kernels' query path with a scale
+ * of 1.  The frequencies are base^(-2i/head_dim), computed as dkv_create does.
+ *   k         device 16-bit (kv_dtype) [num_tiles][16][head_dim] un-rotated key
+ *             rows, 16-byte aligned; row r of tile i sits at position tile_pos[i] + r
+ *   tile_pos  device int32 [num_tiles], each >= 0
+ *   k_out     device fp32 [num_tiles][16][head_dim]: the rotated rows
+ *   q, q_pos, q_out  device fp32 [num_q][head_dim], int32 [num_q], fp32 [num_q][head_dim]
+ *   rope_base > 1; head_dim 64 or 128; k_out, q and q_out 8-byte aligned.
+ * Async on `stream`; allocates nothing.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+DKV_API int dkv_debug_rope(int32_t kv_dtype, int32_t head_dim, double rope_base, const void* k,
+                           const int32_t* tile_pos, int32_t num_tiles, float* k_out, const float* q,
+                           const int32_t* q_pos, int32_t num_q, float* q_out, dkv_stream_t stream);
+
 /* ---- per-kernel timing ---------------------------------------------------
  * dkv_profile_begin -- record CUDA events around every kernel of the next
  * max_calls dkv_attn_decode calls, each on the stream that kernel runs on
@@ -247,6 +305,15 @@ DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const float* q, const
  * created here, never inside dkv_attn_decode.  Not for use while a stream is
  * being captured into a CUDA graph.  Errors: INVALID_ARG, CUDA. */
 DKV_API int dkv_profile_begin(dkv_handle* h, int32_t max_calls);
+
+/* dkv_profile_timeline -- synchronise the handle's device and return, for
+ * recorded call number `call` (0 = the first after dkv_profile_begin), the
+ * start and stop of each kernel in t_ms[6] = {host start, host stop, HBM
+ * start, HBM stop, merge start, merge stop}, in ms from the earliest start
+ * among them; -1 for a kernel that did not run.  Shows whether the host-stream
+ * and HBM kernels overlapped.  Call it before dkv_profile_end.  Errors:
+ * INVALID_ARG (no kernel of that call recorded), CUDA. */
+DKV_API int dkv_profile_timeline(dkv_handle* h, int32_t call, float* t_ms);
 
 /* dkv_profile_end -- synchronise the handle's device, then return in ms[k] the
  * summed device time of kernel k over the recorded calls and in counts[k] how

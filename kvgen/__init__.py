@@ -38,6 +38,8 @@ on its own.
 from __future__ import annotations
 
 import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Iterator
 
 import numpy as np
@@ -169,11 +171,15 @@ def outlier_tokens(w: Workload, b: int, length: int) -> np.ndarray:
     return _rng(w, _OUTLIER, b).random(length) < w.outlier_p
 
 
-def gen_kv_slice(w: Workload, tensor: str, b: int, h: int, length: int, chunk: int = 1 << 22) -> np.ndarray:
-    """Stored bits of K or V for (b, h), tokens 0..length-1: uint16 [length, D]."""
+def gen_kv_slice(w: Workload, tensor: str, b: int, h: int, length: int, chunk: int = 1 << 22,
+                 out: np.ndarray | None = None) -> np.ndarray:
+    """Stored bits of K or V for (b, h), tokens 0..length-1: uint16 [length, D] (written into ``out``
+    when given)."""
     stream = _K if tensor == "k" else _V
     rng = _rng(w, stream, b, h)
-    out = np.empty((length, w.head_dim), dtype=np.uint16)
+    if out is None:
+        out = np.empty((length, w.head_dim), dtype=np.uint16)
+    assert out.shape == (length, w.head_dim) and out.dtype == np.uint16 and out.flags.c_contiguous
     flat = out.reshape(-1)
     n = flat.size
     for s in range(0, n, chunk):
@@ -200,11 +206,23 @@ def gen_kv(w: Workload, seq_lens: np.ndarray | None = None, lmax: int | None = N
     shape = (w.batch, w.num_kv_heads, lmax, w.head_dim)
     k = np.zeros(shape, dtype=np.uint16)
     v = np.zeros(shape, dtype=np.uint16)
-    for b in range(w.batch):
+    # every (tensor, b, h) slice has its own stream, so the slices are drawn on
+    # a thread pool (numpy's generators and ufuncs release the GIL) with
+    # results identical to a serial loop
+    jobs = [(t, b, h) for b in range(w.batch) for h in range(w.num_kv_heads) for t in ("k", "v")]
+
+    def draw(job):
+        t, b, h = job
         L = int(seq_lens[b])
-        for h in range(w.num_kv_heads):
-            k[b, h, :L] = gen_kv_slice(w, "k", b, h, L)
-            v[b, h, :L] = gen_kv_slice(w, "v", b, h, L)
+        gen_kv_slice(w, t, b, h, L, out=(k if t == "k" else v)[b, h, :L])
+
+    workers = max(1, min(len(jobs), len(os.sched_getaffinity(0)), 32))
+    if workers == 1 or k.nbytes < (64 << 20):
+        for j in jobs:
+            draw(j)
+    else:
+        with ThreadPoolExecutor(workers) as pool:
+            list(pool.map(draw, jobs))
     return k, v
 
 

@@ -3,6 +3,8 @@ the CUDA path through the C ABI, and run the fp64 oracle on the same inputs."""
 from __future__ import annotations
 
 import functools
+import json
+import os
 
 import numpy as np
 import torch
@@ -72,3 +74,28 @@ def max_err(got: np.ndarray, want: np.ndarray) -> float:
     assert got.shape == want.shape
     assert np.isfinite(got).all(), "non-finite output"
     return float(np.abs(got.astype(np.float64) - want).max())
+
+
+def record(test: str, workload: str, err: float, groups: str = "all") -> None:
+    """Append one measured parity error to the JSON-lines file named by DKV_PARITY_LOG, if set."""
+    log = os.environ.get("DKV_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"test": test, "workload": workload, "max_abs_err": err, "groups": groups,
+                                "tolerance": TOL}) + "\n")
+
+
+def sampled_groups(w: kvgen.Workload, n: int, seed: int) -> np.ndarray:
+    """uint8 [B, Hkv] mask of n (batch, kv head) groups drawn without replacement."""
+    rng = np.random.default_rng(seed)
+    mask = np.zeros((w.batch, w.num_kv_heads), dtype=np.uint8)
+    for i in rng.choice(w.batch * w.num_kv_heads, size=min(n, w.batch * w.num_kv_heads), replace=False):
+        mask.flat[i] = 1
+    return mask
+
+
+def sampled_err(w: kvgen.Workload, got: np.ndarray, want: np.ndarray, mask: np.ndarray) -> float:
+    """Max abs error over the query-head rows of the masked groups."""
+    rows = np.repeat(mask.astype(bool), w.group_size, axis=1)
+    assert np.isfinite(got[rows]).all(), "non-finite output"
+    return float(np.abs(got[rows].astype(np.float64) - want[rows]).max())

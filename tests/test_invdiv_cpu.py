@@ -55,7 +55,9 @@ def test_invariant_divisor_matches_integer_division(tmp_path):
     src = tmp_path / "invdiv.cu"
     src.write_text(PROGRAM)
     exe = tmp_path / "invdiv"
-    subprocess.run([nvcc, "-O2", "-std=c++17", f"-I{CSRC}", "-o", str(exe), str(src)], check=True,
+    # the header holds sm_100a device code (packed fp32 intrinsics): compile for that target
+    subprocess.run([nvcc, "-O2", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", f"-I{CSRC}", "-o",
+                    str(exe), str(src)], check=True,
                    capture_output=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     tests, bad = map(int, out.stdout.split())

@@ -49,3 +49,17 @@ def test_sweep_has_twenty_cells_with_distinct_seeds():
     cells = kvgen.sweep_cells()
     assert len(cells) == 20 and len({c.seed for c in cells}) == 20
     assert {c.host_fraction for c in cells} == set(kvgen.SWEEP_HOST_FRACTION)
+
+
+def test_threaded_generation_matches_serial_slices():
+    """gen_kv draws large workloads on a thread pool: every slice must equal its serial draw."""
+    w = kvgen.LLAMA3_8B.replace(batch=2, num_kv_heads=4, num_q_heads=16, ctx=(40000, 70000), seed=9)
+    lens = kvgen.gen_seq_lens(w)
+    k, v = kvgen.gen_kv(w, lens)
+    assert k.nbytes >= (64 << 20)   # large enough to take the threaded path
+    for b in range(w.batch):
+        for h in range(w.num_kv_heads):
+            L = int(lens[b])
+            assert np.array_equal(k[b, h, :L], kvgen.gen_kv_slice(w, "k", b, h, L))
+            assert np.array_equal(v[b, h, :L], kvgen.gen_kv_slice(w, "v", b, h, L))
+            assert not k[b, h, L:].any() and not v[b, h, L:].any()
