@@ -58,17 +58,23 @@ struct DeviceGuard {
 };
 
 #ifndef DKV_HOST_STAGES
-#define DKV_HOST_STAGES 4
+#define DKV_HOST_STAGES 3
 #endif
 constexpr int kHostStages = DKV_HOST_STAGES;  // ring depth of the zero-copy host kernel (build-time knob)
 #ifndef DKV_DEV_STAGES
 #define DKV_DEV_STAGES 3
 #endif
 constexpr int kDevStages = DKV_DEV_STAGES;  // ring depth of the HBM kernel (build-time knob)
+// How the HBM kernel moves its tiles (build-time knob): 0 always 16-byte
+// cp.async; 1 (default) tensor copies when it runs beside the zero-copy host
+// kernel and cp.async when it has the GPU to itself; 2 always tensor copies.
+// Beside the host stream the cp.async loads of the HBM kernel slow to less
+// than half speed while the tensor copies keep theirs; alone, cp.async is a
+// few percent faster.
 #ifndef DKV_DEV_TMA
 #define DKV_DEV_TMA 1
 #endif
-constexpr bool kDevTma = DKV_DEV_TMA != 0;  // HBM kernel tiles by tensor copies (else 16-byte cp.async; build-time knob)
+constexpr int kDevTmaMode = DKV_DEV_TMA;
 constexpr int kDefaultHostCtas = 16;
 constexpr int kListThreads = 1024;  // threads of the pool-lists kernel
 
@@ -184,7 +190,7 @@ struct dkv_handle {
   cudaStream_t aux = nullptr;
   cudaEvent_t ev_fork = nullptr;
   cudaEvent_t ev_join = nullptr;
-  SplitEntry host_kernel{}, dev_kernel{}, multi_kernel{};
+  SplitEntry host_kernel{}, dev_kernel{}, dev_tma_kernel{}, multi_kernel{};  // dev: cp.async; dev_tma: tensor copies
   // tensor maps of the last device pool and staging pool the HBM kernel read
   struct PoolMaps {
     const void* k = nullptr;
@@ -272,8 +278,8 @@ int pool_maps(dkv_handle* h, dkv_handle::PoolMaps& cache, const void* k, const v
   if (rows >= (1LL << 31)) return fail(DKV_ERR_INVALID_ARG, "a pool holds 2^31 or more token rows");
   if (cache.k != k || cache.v != v || cache.rows != rows) {
     cache.rows = -1;
-    if (!dkv::encode_pool_map(&cache.maps.k, k, rows, h->cfg.head_dim) ||
-        !dkv::encode_pool_map(&cache.maps.v, v, rows, h->cfg.head_dim))
+    if (!dkv::encode_pool_map(&cache.maps.k, k, rows, h->cfg.head_dim, true) ||
+        !dkv::encode_pool_map(&cache.maps.v, v, rows, h->cfg.head_dim, false))
       return fail(DKV_ERR_CUDA, "cuTensorMapEncodeTiled rejected the pool's tensor map");
     cache.k = k;
     cache.v = v;
@@ -353,7 +359,8 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   h->host_ctas = c.host_ctas > 0 ? c.host_ctas : kDefaultHostCtas;
   const bool rope = c.rope_base > 0.0;
   h->host_kernel = pick_split<kHostStages, false>(c.head_dim, G, bf16, rope);
-  h->dev_kernel = pick_split<kDevStages, kDevTma>(c.head_dim, G, bf16, rope);
+  h->dev_kernel = pick_split<kDevStages, false>(c.head_dim, G, bf16, rope);
+  h->dev_tma_kernel = pick_split<kDevStages, true>(c.head_dim, G, bf16, rope);
   h->multi_kernel = pick_multi(c.head_dim, bf16, c.rope_base > 0.0);
   h->merge = c.head_dim == 64 ? &launch_merge<64, 16> : &launch_merge<128, 8>;
 
@@ -363,7 +370,8 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   };
   cudaError_t e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, c.device);
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaDeviceGetAttribute"));
-  h->beside_host = fits_beside(h->host_kernel.ptr, split_smem(c.head_dim, kHostStages), h->dev_kernel.ptr,
+  h->beside_host = fits_beside(h->host_kernel.ptr, split_smem(c.head_dim, kHostStages),
+                               (kDevTmaMode == 0 ? h->dev_kernel : h->dev_tma_kernel).ptr,
                                split_smem(c.head_dim, kDevStages), c.device);
   h->units_target = static_cast<int>(launch_warps(h, false));
   // partial rows: batch * Tq * Hq * (host splits + device splits), each launch's
@@ -375,12 +383,26 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   e = cudaFuncSetAttribute(h->host_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(split_smem(c.head_dim, kHostStages)));
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(host kernel)"));
-  e = cudaFuncSetAttribute(h->dev_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(split_smem(c.head_dim, kDevStages)));
-  if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(HBM kernel)"));
+  for (const SplitEntry* k : {&h->dev_kernel, &h->dev_tma_kernel}) {
+    e = cudaFuncSetAttribute(k->ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(split_smem(c.head_dim, kDevStages)));
+    if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(HBM kernel)"));
+  }
   e = cudaFuncSetAttribute(h->multi_kernel.ptr, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(multi_smem(c.head_dim)));
   if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(multi-token kernel)"));
+  // every kernel of a step prefers the largest shared-memory carveout, so an SM
+  // need not change its L1/shared split between the step's kernels
+  {
+    const void* all[] = {h->host_kernel.ptr, h->dev_kernel.ptr, h->dev_tma_kernel.ptr, h->multi_kernel.ptr,
+                         reinterpret_cast<const void*>(&dkv::lists_kernel<kListThreads>),
+                         reinterpret_cast<const void*>(c.head_dim == 64 ? &dkv::merge_kernel<64, 16>
+                                                                         : &dkv::merge_kernel<128, 8>)};
+    for (const void* f : all) {
+      e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(carveout)"));
+    }
+  }
   int nalloc = 0;
   const bool armed = g_fail_alloc > 0;
   if (dev_alloc(reinterpret_cast<void**>(&h->part_o), h->part_rows * c.head_dim * sizeof(float), &nalloc) ||
@@ -547,8 +569,10 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
     dkv::set_divisors(lp);
     return lp;
   };
+  const bool dev_tma = !multi && (kDevTmaMode == 2 || (kDevTmaMode == 1 && concurrent));
   const SplitEntry& host_k = multi ? h->multi_kernel : h->host_kernel;
-  const SplitEntry& dev_k = multi ? h->multi_kernel : h->dev_kernel;
+  const SplitEntry& dev_k = multi ? h->multi_kernel : (dev_tma ? h->dev_tma_kernel : h->dev_kernel);
+  const SplitEntry& stage_k = multi ? h->multi_kernel : (kDevTmaMode == 2 ? h->dev_tma_kernel : h->dev_kernel);
   const size_t host_smem = multi ? multi_smem(c.head_dim) : split_smem(c.head_dim, kHostStages);
   const size_t dev_smem = multi ? multi_smem(c.head_dim) : split_smem(c.head_dim, kDevStages);
   auto ctas_for = [&](const dkv::SplitParams& lp, int cap) {
@@ -590,8 +614,9 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
     hp.id_lo = 0;
     hp.id_hi = host_split;
     const dkv::TileMaps* maps = &no_maps;
-    if (!multi && (rc = pool_maps(h, h->stage_maps, k_stage, v_stage, host_split, &maps)) != DKV_OK) return rc;
-    dev_k.fn(dim3(ctas_for(hp, 2 * h->sm_count)), dev_smem, s, hp, *maps);
+    if (!multi && kDevTmaMode == 2 && (rc = pool_maps(h, h->stage_maps, k_stage, v_stage, host_split, &maps)) != DKV_OK)
+      return rc;
+    stage_k.fn(dim3(ctas_for(hp, 2 * h->sm_count)), dev_smem, s, hp, *maps);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 0, s, true)) != DKV_OK) return rc;
     ++launches;
@@ -616,12 +641,12 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
     dp.v_pool = static_cast<const uint16_t*>(v_dev);
     dp.id_lo = host_split;
     dp.id_hi = host_split + num_dev_blocks;
-    if (!multi && g_stall_copy) {
+    if (dev_tma && g_stall_copy) {
       dp.stall_first_copy = 1;
       g_stall_copy = 0;
     }
     const dkv::TileMaps* maps = &no_maps;
-    if (!multi && num_dev_blocks > 0 &&
+    if (dev_tma && num_dev_blocks > 0 &&
         (rc = pool_maps(h, h->dev_maps, k_dev, v_dev, num_dev_blocks, &maps)) != DKV_OK)
       return rc;
     if ((rc = prof_mark(h, 1, s, false)) != DKV_OK) return rc;

@@ -159,17 +159,19 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// ---- tile copies by the tensor memory accelerator (HBM launch)
+// ---- shared-memory tiles and the tensor copies that can fill them
 //
-// A K or V tile (16 token rows of D 16-bit elements) arrives as D/64 boxes of
-// 16 rows x 64 elements (128 bytes per row) with the 128-byte swizzle: inside
-// each 1024-byte group of 8 rows, 16-byte chunk c of row r lands at chunk
-// c ^ (r mod 8).  tile_off gives that layout for every producer (the tensor
-// copies of the HBM launch, the 16-byte cp.async of the host launch) and
-// every consumer (the score and PV loops), so 8 lanes that read one row, and
-// the 8 rows of one ldmatrix phase, each touch 8 distinct bank groups.
+// A K tile (16 token rows of D 16-bit elements) is stored as it comes, row
+// after row: the 8 lanes of a token group read one row's 8 chunks.  A V tile
+// is stored as D/64 sub-tiles of 16 rows x 128 bytes with the 128-byte
+// swizzle: inside each 1024-byte group of 8 rows, 16-byte chunk c of row r
+// lands at chunk c ^ (r mod 8), so the 8 rows of one ldmatrix phase touch 8
+// distinct bank groups.  tile_off gives that V layout to every producer (the
+// 16-byte cp.async, the tensor copies) and to the PV loop.
 
-// Tensor maps of the K and V pools of one launch (unused by cp.async launches).
+// Tensor maps of the K pool (boxes of 16 plain rows) and the V pool (boxes
+// of 16 rows x 64 elements, 128-byte swizzle) of one launch; unused by
+// cp.async launches.
 struct TileMaps {
   CUtensorMap k, v;
 };
@@ -717,6 +719,14 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p, co
     const int e = lane + 32 * k;
     dofs[k] = tile_off(e / CPR, e % CPR);
   }
+  // ldmatrix offsets of this lane inside a V tile: row (lane & 15), chunk
+  // 2 qd + (lane >> 4); chunks c and c + 8 differ by the 2048-byte half, so
+  // four values cover qd = 0..D/16-1.
+  int vofs_q[4];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) vofs_q[q4] = tile_off((lane & 7) | (lane & 8), 2 * q4 + (lane >> 4));
+  // test hook (dkv_debug_stall_copy): the first tile copy of warp 0 of CTA 0 is left unissued
+  bool stall_next = TMA && p.stall_first_copy && blockIdx.x == 0 && warp == 0;
   uint32_t phase = 0;     // per stage: parity of its next completion (TMA)
   uint32_t inflight = 0;  // per stage: tensor copies issued and not yet waited for (TMA)
   bool broken = false;    // a copy did not complete in time: no more copies, every later tile poisoned (TMA)
@@ -733,33 +743,40 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p, co
         const uint32_t bar = smem_u32(&tail.bar[warp][slot]);
         if (copy) {
           const int row0 = (d.pidx * p.hkv + h) * p.block_size + sub * kTileTokens;
-          fence_proxy_async();
           mbar_arrive_expect_tx(bar, 2 * TILE);
-          // the test hook leaves this one stage armed with nothing to complete it
-          const bool stall = p.stall_first_copy && blockIdx.x == 0 && warp == 0 && inflight == 0 && phase == 0;
-          if (!stall) {
+          // the test hook leaves one stage armed with nothing to complete it
+          if (!stall_next) {
+            tma_load_2d(smem_u32(sk), &maps.k, 0, row0, bar);   // K: one box of 16 plain rows
 #pragma unroll
-            for (int x = 0; x < D / 64; ++x) {
-              tma_load_2d(smem_u32(sk + x * kTileTokens * 128), &maps.k, 64 * x, row0, bar);
+            for (int x = 0; x < D / 64; ++x)                    // V: D/64 swizzled 64-element halves
               tma_load_2d(smem_u32(sv + x * kTileTokens * 128), &maps.v, 64 * x, row0, bar);
-            }
           }
         } else {
           mbar_arrive(bar);
         }
       }
-      if (copy) inflight |= 1u << slot;
+      if (copy) {
+        inflight |= 1u << slot;
+        stall_next = false;
+      }
     } else {
       if (!copy) return;
       const size_t row0 = (static_cast<size_t>(d.pidx) * p.hkv + h) * p.block_size + sub * kTileTokens;
       const char* gk = reinterpret_cast<const char*>(p.k_pool + row0 * D) + lane * 16;
       const char* gv = reinterpret_cast<const char*>(p.v_pool + row0 * D) + lane * 16;
+      if (nvalid == kTileTokens) {
 #pragma unroll
-      for (int k = 0; k < KCOPIES; ++k) {
-        const int o = dofs[k & 3] + (k >> 2) * 1024;
-        const int nb = (nvalid == kTileTokens || (lane + 32 * k) / CPR < nvalid) ? 16 : 0;
-        cp_async16(sk + o, nb ? gk + 512 * k : gk - lane * 16, nb);
-        cp_async16(sv + o, nb ? gv + 512 * k : gv - lane * 16, nb);
+        for (int k = 0; k < KCOPIES; ++k) {
+          cp_async16(sk + lane * 16 + 512 * k, gk + 512 * k, 16);
+          cp_async16(sv + dofs[k & 3] + (k >> 2) * 1024, gv + 512 * k, 16);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < KCOPIES; ++k) {
+          const int nb = (lane + 32 * k) / CPR < nvalid ? 16 : 0;   // rows past the end: zeros, nothing read
+          cp_async16(sk + lane * 16 + 512 * k, nb ? gk + 512 * k : gk - lane * 16, nb);
+          cp_async16(sv + dofs[k & 3] + (k >> 2) * 1024, nb ? gv + 512 * k : gv - lane * 16, nb);
+        }
       }
     }
   };
@@ -898,12 +915,10 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p, co
     float v[4 * G];  // partial scores, index g * 4 + m
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const int t = tg + 4 * m;
       float2 X[NP2], Y[NP2];
-      constexpr int XB = 0, YB = D;            // byte offsets of the row's two halves
-      const int xb = XB + li * PPL * 2, yb = YB + li * PPL * 2;
-      load_pairs<NP2, BF16>(sk + tile_off(t, xb >> 4) + (xb & 15), X);
-      load_pairs<NP2, BF16>(sk + tile_off(t, yb >> 4) + (yb & 15), Y);
+      const char* krow = sk + (tg + 4 * m) * ROW + li * PPL * 2;   // K rows are stored as they come
+      load_pairs<NP2, BF16>(krow, X);
+      load_pairs<NP2, BF16>(krow + D, Y);
       if constexpr (ROPE) rope_rotate_advance<NP2>(X, Y, C, S, re, rf);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -1001,11 +1016,10 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p, co
       a[0] = lane < 16 ? ha : la;
       a[1] = lane < 16 ? hb : lb;
     }
-    const int vrow = (lane & 7) | (lane & 8);
 #pragma unroll
     for (int qd = 0; qd < D / 16; ++qd) {
       uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(sv + tile_off(vrow, 2 * qd + (lane >> 4)), b0, b1, b2, b3);
+      ldsm_x4_t(sv + vofs_q[qd & 3] + (qd >> 2) * (kTileTokens * 128), b0, b1, b2, b3);
       mma16816_top<BF16>(acc[2 * qd], a, b0, b1);
       mma16816_top<BF16>(acc[2 * qd + 1], a, b2, b3);
     }

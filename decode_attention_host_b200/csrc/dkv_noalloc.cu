@@ -35,17 +35,20 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[DKV_NOALLOC_SCR
 
 constexpr int kMaxDevices = 64;
 #ifndef DKV_HOST_STAGES
-#define DKV_HOST_STAGES 4
+#define DKV_HOST_STAGES 3
 #endif
 constexpr int kHostStages = DKV_HOST_STAGES;
 #ifndef DKV_DEV_STAGES
 #define DKV_DEV_STAGES 3
 #endif
 constexpr int kDevStages = DKV_DEV_STAGES;
+// HBM-kernel copy path, as in dkv_api.cu: here the split kernels run one
+// after the other, never beside each other, so tensor copies are used only
+// when the knob asks for them always (2).
 #ifndef DKV_DEV_TMA
 #define DKV_DEV_TMA 1
 #endif
-constexpr bool kDevTma = DKV_DEV_TMA != 0;
+constexpr bool kDevTma = DKV_DEV_TMA == 2;
 constexpr int kHostCtas = 16;
 constexpr int kListThreads = 1024;
 constexpr size_t kStatusOffset = 0;     // int32 status word
@@ -240,11 +243,12 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
     return set_error(DKV_ERR_INVALID_ARG, "dkv_attn_decode_noalloc: device pools must be memory of cfg->device");
   // tensor maps of the device pool for the HBM kernel's tile copies (host-side encoding, no allocation)
   dkv::TileMaps maps{};
-  if (num_dev_blocks > 0) {
+  if (kDevTma && num_dev_blocks > 0) {
     const long long rows = static_cast<long long>(num_dev_blocks) * c.num_kv_heads * c.block_size;
     if (rows >= (1LL << 31))
       return set_error(DKV_ERR_INVALID_ARG, "dkv_attn_decode_noalloc: a pool holds 2^31 or more token rows");
-    if (!dkv::encode_pool_map(&maps.k, k_dev, rows, c.head_dim) || !dkv::encode_pool_map(&maps.v, v_dev, rows, c.head_dim))
+    if (!dkv::encode_pool_map(&maps.k, k_dev, rows, c.head_dim, true) ||
+        !dkv::encode_pool_map(&maps.v, v_dev, rows, c.head_dim, false))
       return set_error(DKV_ERR_CUDA, "dkv_attn_decode_noalloc: cuTensorMapEncodeTiled rejected the pool's tensor map");
   }
 

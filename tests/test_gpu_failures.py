@@ -90,7 +90,8 @@ def test_a_copy_that_never_completes_times_out_and_is_reported():
     rows for the units it held; the other rows are exact and the next call is clean."""
     import time
     import oracle
-    w = kvgen.LLAMA3_8B.replace(name="stall", batch=2, ctx=3000, seed=72, host_fraction=0.0)
+    # blocks in both pools: the HBM kernel runs beside the host kernel and moves its tiles by tensor copies
+    w = kvgen.LLAMA3_8B.replace(name="stall", batch=2, ctx=3000, seed=72, host_fraction=0.5)
     case = gc.Case(w)
     want = case.oracle()
     dkv.dkv_debug_stall_copy(True)
