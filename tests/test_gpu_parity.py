@@ -25,7 +25,7 @@ def check(case: gc.Case, tol=gc.TOL, test: str = "parity"):
 
 def test_tiny_gqa_matches_oracle_and_golden():
     case = gc.Case(kvgen.TINY_GQA)
-    got, err = check(case)
+    got, err = check(case, test="test_tiny_gqa_matches_oracle_and_golden")
     _, golden = load_golden()
     assert np.abs(got[0] - golden).max() <= gc.TOL
     # tokens 0..255 on the host, 256..511 in HBM: the pool lists, both split kernels and the merge ran
@@ -43,7 +43,7 @@ def test_tiny_gqa_matches_oracle_and_golden():
 def test_reduced_workloads(name, kw):
     base = kvgen.get(name.replace("_norope", ""))
     case = gc.Case(base.replace(**kw))
-    check(case)
+    check(case, test="test_reduced_workloads")
     case.free()
 
 
@@ -65,7 +65,7 @@ def test_sweep_4k_cells_full_size(f):
 def test_every_head_shape_and_dtype(d, g, dt):
     w = kvgen.LLAMA3_8B.replace(name=f"shape_d{d}_g{g}", batch=3, num_kv_heads=2, num_q_heads=2 * g, head_dim=d,
                                 kv_dtype=dt, ctx=(1, 700), block_size=32, seed=40 + d + g)
-    check(gc.Case(w))
+    check(gc.Case(w), test="test_every_head_shape_and_dtype")
 
 
 def test_edge_lengths_in_one_batch():
@@ -73,7 +73,7 @@ def test_edge_lengths_in_one_batch():
     lens = [0, 1, 15, 16, 17, 31, 32, 33, 64, 1000]
     w = kvgen.LLAMA3_8B.replace(name="edges", batch=len(lens), ctx=max(lens), seed=77)
     case = gc.Case(w, lens=lens)
-    got, _ = check(case)
+    got, _ = check(case, test="test_edge_lengths_in_one_batch")
     assert not got[0].any(), "an empty sequence must give a zero row"
     case.free()
 
@@ -272,7 +272,7 @@ def test_large_blocks(block_size, d, placement):
         w = kvgen.LLAMA3_8B.replace(name=f"blocks_s{block_size}_d{d}", batch=3, head_dim=d, ctx=(700, 5000),
                                     block_size=block_size, placement=placement, host_fraction=0.5, seed=block_size + d)
     case = gc.Case(w)
-    check(case)
+    check(case, test="test_large_blocks")
     if w.name == "tiny_s256":
         assert case.kv.host_split == 1 and case.kv.num_dev_blocks == 1
     case.free()
