@@ -63,3 +63,21 @@ def test_reference_arm_prints_one_json_line():
     assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] == 2
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["config"]["workload"] == "tiny_gqa"
+
+
+def test_reduced_context_keeps_the_shape_and_renames_the_workload():
+    w = bench.workload_for_rank("long_ctx", 0, 262144)
+    base = bench.workload_for_rank("long_ctx", 0)
+    assert w.name == "long_ctx_ctx262144" and w.ctx == 262144
+    assert (w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.placement, w.host_fraction) == \
+        (base.batch, base.num_q_heads, base.num_kv_heads, base.head_dim, base.block_size, base.placement,
+         base.host_fraction)
+    assert bench.workload_for_rank("long_ctx", 2, 4096).seed == base.seed + 2000
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    args = bench.parse_args([])
+    assert args.workload == "long_ctx" and args.mode == "zero_copy" and args.gpus == 1
+    import kvgen
+    sizes = {n: kvgen.get(n).batch * kvgen.get(n).max_ctx for n in ("tiny_gqa", "llama3_8b", "long_ctx", "opt_6_7b")}
+    assert max(sizes, key=sizes.get) == "long_ctx"
