@@ -102,7 +102,7 @@ struct SplitParams {
   int32_t n_units;          // B * nsplit * Hkv
   int32_t rope;             // 0: no rotation
   float qscale;             // softmax scale * log2(e)
-  int32_t stall_first_copy; // test hook: warp 0 of CTA 0 arms its first tile's barrier but issues no copy
+  int32_t stall_first_copy; // test hook: the first tile of unit 0 arms its barrier but issues no copy
   int32_t extra_tokens;     // tokens past seq_lens that belong to the unit (multi-token queries: Tq - 1)
   int32_t num_queries;      // query tokens per sequence (1 for decode)
   InvDiv div_hkv, div_nsplit, div_bs;  // hkv, nsplit, block_size (set_divisors)
@@ -725,8 +725,10 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p, co
   int vofs_q[4];
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4) vofs_q[q4] = tile_off((lane & 7) | (lane & 8), 2 * q4 + (lane >> 4));
-  // test hook (dkv_debug_stall_copy): the first tile copy of warp 0 of CTA 0 is left unissued
-  bool stall_next = TMA && p.stall_first_copy && blockIdx.x == 0 && warp == 0;
+  // test hook (dkv_debug_stall_copy): the first tile copy of unit 0 is left
+  // unissued.  Units are handed out once each, so exactly one warp of the
+  // launch meets it, whichever CTA runs first.
+  bool stall_armed = TMA && p.stall_first_copy;
   uint32_t phase = 0;     // per stage: parity of its next completion (TMA)
   uint32_t inflight = 0;  // per stage: tensor copies issued and not yet waited for (TMA)
   bool broken = false;    // a copy did not complete in time: no more copies, every later tile poisoned (TMA)
@@ -745,7 +747,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p, co
           const int row0 = (d.pidx * p.hkv + h) * p.block_size + sub * kTileTokens;
           mbar_arrive_expect_tx(bar, 2 * TILE);
           // the test hook leaves one stage armed with nothing to complete it
-          if (!stall_next) {
+          if (!(stall_armed && d.unit == 0)) {
             tma_load_2d(smem_u32(sk), &maps.k, 0, row0, bar);   // K: one box of 16 plain rows
 #pragma unroll
             for (int x = 0; x < D / 64; ++x)                    // V: D/64 swizzled 64-element halves
@@ -757,7 +759,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p, co
       }
       if (copy) {
         inflight |= 1u << slot;
-        stall_next = false;
+        if (d.unit == 0) stall_armed = false;
       }
     } else {
       if (!copy) return;

@@ -271,10 +271,11 @@ DKV_API int dkv_debug_fail_alloc(int32_t nth);
 /* dkv_debug_stall_copy -- TEST ONLY: in the next dkv_attn_decode on the
  * calling thread whose HBM kernel moves its tiles with tensor copies (a call
  * with blocks in both pools, where that kernel runs beside the zero-copy host
- * kernel), warp 0 of its first CTA arms
- * the barrier of its first tile copy but issues no copy, so its bounded wait
- * runs out (about 2 s): the call must then report DKV_STATUS_COPY_TIMEOUT,
- * write NaN for that warp's units and leave the device usable.  The hook is
+ * kernel), the warp that takes that kernel's first work unit arms the
+ * barrier of the unit's first tile copy but issues no copy, so its bounded
+ * wait runs out (about 2 s): the call must then report
+ * DKV_STATUS_COPY_TIMEOUT, write NaN for that warp's units and leave the
+ * device usable.  The hook is
  * cleared by that call; 0 disarms it.  Always returns DKV_OK. */
 DKV_API int dkv_debug_stall_copy(int32_t enable);
 
