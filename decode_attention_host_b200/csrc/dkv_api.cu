@@ -153,20 +153,20 @@ size_t multi_smem(int D) { return static_cast<size_t>(dkv::kWarps) * 5 * dkv::kT
 // The merge, optionally as a programmatic dependent launch of the split kernel
 // just before it on the stream: its grid is set up while that kernel drains
 // and its first instruction waits for that kernel's results.
-using MergeFn = cudaError_t (*)(dim3, size_t, cudaStream_t, const dkv::MergeParams&, bool);
-template <int D, int NG>
-cudaError_t launch_merge(dim3 grid, size_t smem, cudaStream_t s, const dkv::MergeParams& p, bool dependent) {
+using MergeFn = cudaError_t (*)(int, cudaStream_t, const dkv::MergeParams&, bool);
+template <int D>
+cudaError_t launch_merge(int rows, cudaStream_t s, const dkv::MergeParams& p, bool dependent) {
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(NG * D);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(rows);
+  cfg.blockDim = dim3(32 * dkv::merge_warps(p.nslots, D));
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = dependent ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, dkv::merge_kernel<D, NG>, p);
+  return cudaLaunchKernelEx(&cfg, dkv::merge_kernel<D>, p);
 }
 
 }  // namespace
@@ -362,7 +362,7 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   h->dev_kernel = pick_split<kDevStages, false>(c.head_dim, G, bf16, rope);
   h->dev_tma_kernel = pick_split<kDevStages, true>(c.head_dim, G, bf16, rope);
   h->multi_kernel = pick_multi(c.head_dim, bf16, c.rope_base > 0.0);
-  h->merge = c.head_dim == 64 ? &launch_merge<64, 16> : &launch_merge<128, 8>;
+  h->merge = c.head_dim == 64 ? &launch_merge<64> : &launch_merge<128>;
 
   auto bail = [&](int code) {
     release(h);
@@ -396,8 +396,8 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   {
     const void* all[] = {h->host_kernel.ptr, h->dev_kernel.ptr, h->dev_tma_kernel.ptr, h->multi_kernel.ptr,
                          reinterpret_cast<const void*>(&dkv::lists_kernel<kListThreads>),
-                         reinterpret_cast<const void*>(c.head_dim == 64 ? &dkv::merge_kernel<64, 16>
-                                                                         : &dkv::merge_kernel<128, 8>)};
+                         reinterpret_cast<const void*>(c.head_dim == 64 ? &dkv::merge_kernel<64>
+                                                                         : &dkv::merge_kernel<128>)};
     for (const void* f : all) {
       e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
       if (e != cudaSuccess) return bail(cuda_fail(e, "cudaFuncSetAttribute(carveout)"));
@@ -668,7 +668,7 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   mp.has_host = run_host;
   mp.has_dev = run_dev;
   if ((rc = prof_mark(h, 2, s, false)) != DKV_OK) return rc;
-  DKV_CUDA(h->merge(dim3(batch * nq * c.num_q_heads), nslots * sizeof(float), s, mp, merge_follows_split));
+  DKV_CUDA(h->merge(batch * nq * c.num_q_heads, s, mp, merge_follows_split));
   if ((rc = prof_mark(h, 2, s, true)) != DKV_OK) return rc;
   ++launches;
   h->last_launches = launches;

@@ -1147,75 +1147,99 @@ __global__ void __launch_bounds__(32) rope_debug_kernel(const __grid_constant__ 
 
 // ----------------------------------------------------------------------------- merge kernel
 
-// One CTA per (b, hq); blockDim = NG * D threads: NG slot groups x D dims.
-template <int D, int NG>
-__global__ void __launch_bounds__(NG * D) merge_kernel(const MergeParams p) {
-  extern __shared__ float wts[];  // [nslots]
-  __shared__ float red_m[NG * D / 32], red_z[NG * D / 32];
-  __shared__ int red_nan[NG * D / 32];
-  __shared__ float part[NG][D];
+// One CTA per output row (b, hq); blockDim = 32 * W threads, W = the slot
+// warps (merge_warps).  Warp w takes slots w, w + W, ... and keeps its own
+// online combine of them: a running max m_w, sum z_w = sum 2^(lse_i - m_w)
+// and acc_w = sum 2^(lse_i - m_w) o_i for its lane's D/32 dims, so the lse
+// and the partial outputs are read in one pass.  After one barrier the first
+// D threads rescale the warps' results to the row's max and divide.  A NaN
+// slot makes the row NaN; a row with no valid non-empty slot is zero.
+constexpr int kMergeMaxWarps = 32;
+
+// slot warps of a merge CTA: one per slot up to 32, at least D/32 for the
+// final combine
+__host__ __device__ constexpr int merge_warps(int nslots, int D) {
+  return nslots >= kMergeMaxWarps ? kMergeMaxWarps : (nslots > D / 32 ? nslots : D / 32);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(const MergeParams p) {
+  constexpr int V = D / 32;  // dims per lane
+  static_assert(V == 2 || V == 4, "head_dim 64 or 128");
+  __shared__ float s_acc[kMergeMaxWarps][D];
+  __shared__ float s_m[kMergeMaxWarps], s_z[kMergeMaxWarps];
+  __shared__ int s_nan[kMergeMaxWarps];
   // launched as a programmatic dependent of the split kernel: wait until that
   // grid has completed and its partials are visible (no-op otherwise)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int row = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
   const float* lse = p.part_lse + static_cast<size_t>(row) * p.nslots;
-  const float* o = p.part_o + static_cast<size_t>(row) * p.nslots * D;
-  auto valid = [&](int i) { return i < p.nsplit ? p.has_host != 0 : p.has_dev != 0; };
+  const float* o = p.part_o + static_cast<size_t>(row) * p.nslots * D + lane * V;
 
-  float mx = -INFINITY;
-  int nan = 0;
-  for (int i = tid; i < p.nslots; i += NG * D) {
-    if (!valid(i)) continue;
-    const float v = lse[i];
-    nan |= isnan(v) ? 1 : 0;
-    mx = fmaxf(mx, v);
-  }
-  for (int off = 16; off > 0; off >>= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-    nan |= __shfl_xor_sync(kFull, nan, off);
-  }
-  if ((tid & 31) == 0) { red_m[tid >> 5] = mx; red_nan[tid >> 5] = nan; }
-  __syncthreads();
-  mx = -INFINITY;
-  nan = 0;
+  float m = -INFINITY, z = 0.f;
+  float acc[V];
 #pragma unroll
-  for (int i = 0; i < NG * D / 32; ++i) { mx = fmaxf(mx, red_m[i]); nan |= red_nan[i]; }
-
+  for (int k = 0; k < V; ++k) acc[k] = 0.f;
+  int nan = 0;
+#pragma unroll 2
+  for (int i = warp; i < p.nslots; i += nw) {
+    if (!(i < p.nsplit ? p.has_host : p.has_dev)) continue;
+    const float l = lse[i];
+    float x[V];
+    if constexpr (V == 4) {
+      const float4 t = *reinterpret_cast<const float4*>(o + static_cast<size_t>(i) * D);
+      x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+    } else {
+      const float2 t = *reinterpret_cast<const float2*>(o + static_cast<size_t>(i) * D);
+      x[0] = t.x; x[1] = t.y;
+    }
+    if (isnan(l)) {
+      nan = 1;
+      continue;
+    }
+    if (l == -INFINITY) continue;  // empty split
+    if (l > m) {
+      const float r = exp2f(m - l);  // 0 while m is -inf
+      z *= r;
+#pragma unroll
+      for (int k = 0; k < V; ++k) acc[k] *= r;
+      m = l;
+    }
+    const float w = exp2f(l - m);
+    z += w;
+#pragma unroll
+    for (int k = 0; k < V; ++k) acc[k] = fmaf(w, x[k], acc[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < V; ++k) s_acc[warp][lane * V + k] = acc[k];
+  if (lane == 0) {
+    s_m[warp] = m;
+    s_z[warp] = z;
+    s_nan[warp] = nan;
+  }
+  __syncthreads();
+  if (threadIdx.x >= D) return;
+  // thread d: lane w of its warp holds slot warp w's rescale factor
+  const float mw = lane < nw ? s_m[lane] : -INFINITY;
+  const int anynan = __any_sync(kFull, lane < nw && s_nan[lane] != 0);
+  float M = mw;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
   float* dst = p.out + static_cast<size_t>(row) * D;
-  if (nan || mx == -INFINITY) {
-    if (tid < D) dst[tid] = nan ? __int_as_float(0x7fc00000) : 0.f;
+  const int d = threadIdx.x;
+  if (anynan || M == -INFINITY) {
+    dst[d] = anynan ? __int_as_float(0x7fc00000) : 0.f;
     return;
   }
-  float z = 0.f;
-  for (int i = tid; i < p.nslots; i += NG * D) {
-    const float wi = valid(i) ? exp2f(lse[i] - mx) : 0.f;
-    wts[i] = wi;
-    z += wi;
-  }
-  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFull, z, off);
-  if ((tid & 31) == 0) red_z[tid >> 5] = z;
-  __syncthreads();
-  z = 0.f;
+  const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
+  float Z = lane < nw ? s_z[lane] * sc : 0.f;
 #pragma unroll
-  for (int i = 0; i < NG * D / 32; ++i) z += red_z[i];
-
-  const int d = tid % D;
-  const int grp = tid / D;
-  float acc = 0.f;
-#pragma unroll 2
-  for (int i = grp; i < p.nslots; i += NG) {
-    const float wi = wts[i];
-    if (wi != 0.f) acc = fmaf(wi, o[static_cast<size_t>(i) * D + d], acc);
-  }
-  part[grp][d] = acc;
-  __syncthreads();
-  if (tid < D) {
-    float t = 0.f;
-#pragma unroll
-    for (int g = 0; g < NG; ++g) t += part[g][tid];
-    dst[tid] = t / z;
-  }
+  for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(kFull, Z, off);
+  float a = 0.f;
+  for (int w = 0; w < nw; ++w) a = fmaf(__shfl_sync(kFull, sc, w), s_acc[w][d], a);
+  dst[d] = a / Z;
 }
 
 }  // namespace dkv

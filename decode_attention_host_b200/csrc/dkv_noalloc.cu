@@ -114,19 +114,19 @@ __global__ void noalloc_init_kernel(const __grid_constant__ dkv::RopeFreqs fr, u
   if (i < 4) reinterpret_cast<int32_t*>(base + kWorkOffset)[i] = 0;
 }
 
-template <int D, int NG>
-cudaError_t launch_merge(int rows, size_t smem, cudaStream_t s, const dkv::MergeParams& p, bool dependent) {
+template <int D>
+cudaError_t launch_merge(int rows, cudaStream_t s, const dkv::MergeParams& p, bool dependent) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(rows);
-  cfg.blockDim = dim3(NG * D);
-  cfg.dynamicSmemBytes = smem;
+  cfg.blockDim = dim3(32 * dkv::merge_warps(p.nslots, D));
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = dependent ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, dkv::merge_kernel<D, NG>, p);
+  return cudaLaunchKernelEx(&cfg, dkv::merge_kernel<D>, p);
 }
 
 int cuda_error(cudaError_t e, const char* what) {
@@ -372,8 +372,7 @@ extern "C" DKV_API int dkv_attn_decode_noalloc(const dkv_config* cfg, const floa
   mp.has_host = run_host;
   mp.has_dev = run_dev;
   const int merge_rows = batch * c.num_q_heads;
-  e = D == 64 ? launch_merge<64, 16>(merge_rows, nslots * sizeof(float), s, mp, run_dev)
-              : launch_merge<128, 8>(merge_rows, nslots * sizeof(float), s, mp, run_dev);
+  e = D == 64 ? launch_merge<64>(merge_rows, s, mp, run_dev) : launch_merge<128>(merge_rows, s, mp, run_dev);
   if (e != cudaSuccess) return cuda_error(e, "merge kernel launch");
   if (status_out &&
       (e = cudaMemcpyAsync(status_out, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
