@@ -75,6 +75,24 @@ constexpr int kDevStages = DKV_DEV_STAGES;  // ring depth of the HBM kernel (bui
 #define DKV_DEV_TMA 1
 #endif
 constexpr int kDevTmaMode = DKV_DEV_TMA;
+// How the zero-copy host kernel reads the mapped host pools (build-time
+// knob): 0 (default) 16-byte cp.async; 1 tensor copies through tensor maps
+// over the host pools.  Both reach the same share of the PCIe copy-engine
+// rate (about 0.92); the link, not the SM's load path, sets it.
+#ifndef DKV_HOST_TMA
+#define DKV_HOST_TMA 0
+#endif
+constexpr bool kHostTma = DKV_HOST_TMA != 0;
+// Units per resident warp the single-token HBM kernel's split plan aims at
+// when that kernel has the GPU to itself (build-time knob, 1 to 4; the
+// partial-row workspace covers up to 4).  More, smaller units balance the
+// SMs better but add a query load, RoPE seeds and a partial write per unit;
+// 1 is the fastest measured.
+#ifndef DKV_DEV_OVERSUB
+#define DKV_DEV_OVERSUB 1
+#endif
+constexpr int kDevOversub = DKV_DEV_OVERSUB;
+static_assert(kDevOversub >= 1 && kDevOversub <= 4, "DKV_DEV_OVERSUB must be 1..4");
 constexpr int kDefaultHostCtas = 16;
 constexpr int kListThreads = 1024;  // threads of the pool-lists kernel
 
@@ -197,7 +215,7 @@ struct dkv_handle {
     const void* v = nullptr;
     long long rows = -1;
     dkv::TileMaps maps{};
-  } dev_maps, stage_maps;
+  } dev_maps, stage_maps, host_maps;
   MergeFn merge = nullptr;
   const void* ok_host[2] = {nullptr, nullptr};
   const void* ok_dev[4] = {nullptr, nullptr, nullptr, nullptr};
@@ -358,7 +376,7 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   h->qscale = static_cast<float>(scale * 1.4426950408889634);  // * log2(e)
   h->host_ctas = c.host_ctas > 0 ? c.host_ctas : kDefaultHostCtas;
   const bool rope = c.rope_base > 0.0;
-  h->host_kernel = pick_split<kHostStages, false>(c.head_dim, G, bf16, rope);
+  h->host_kernel = pick_split<kHostStages, kHostTma>(c.head_dim, G, bf16, rope);
   h->dev_kernel = pick_split<kDevStages, false>(c.head_dim, G, bf16, rope);
   h->dev_tma_kernel = pick_split<kDevStages, true>(c.head_dim, G, bf16, rope);
   h->multi_kernel = pick_multi(c.head_dim, bf16, c.rope_base > 0.0);
@@ -528,7 +546,8 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   const long per = static_cast<long>(batch) * c.num_kv_heads;
   const long host_warps = staged ? launch_warps(h, false) : static_cast<long>(dkv::kWarps) * h->host_ctas;
   const dkv::SplitPlan ph = dkv::plan_split(nblk_cap, per, c.block_size, host_warps, 0);
-  const dkv::SplitPlan pd = dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, concurrent), 0);
+  const dkv::SplitPlan pd =
+      dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, concurrent) * (concurrent || multi ? 1 : kDevOversub), 0);
   const int nsplit_h = run_host ? ph.nsplit : 0;
   const int nsplit_d = run_dev ? pd.nsplit : 0;
   const int nslots = nsplit_h + nsplit_d;
@@ -628,8 +647,11 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
     hp.v_pool = static_cast<const uint16_t*>(v_host);
     hp.id_lo = 0;
     hp.id_hi = host_split;
+    const dkv::TileMaps* hmaps = &no_maps;
+    if (kHostTma && !multi && (rc = pool_maps(h, h->host_maps, k_host, v_host, host_split, &hmaps)) != DKV_OK)
+      return rc;
     if ((rc = prof_mark(h, 0, h->aux, false)) != DKV_OK) return rc;
-    host_k.fn(dim3(ctas_for(hp, h->host_ctas)), host_smem, h->aux, hp, no_maps);
+    host_k.fn(dim3(ctas_for(hp, h->host_ctas)), host_smem, h->aux, hp, *hmaps);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 0, h->aux, true)) != DKV_OK) return rc;
     DKV_CUDA(cudaEventRecord(h->ev_join, h->aux));
