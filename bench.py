@@ -11,11 +11,11 @@ host memory and the newest 10% in HBM: 4 GiB of KV per step).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dkv|reference]
                     [--mode zero_copy|staged|planned] [--hbm-budget-frac F]
 
---mode planned measures the workload at its own placement first, gives the
-host-stream and HBM kernels' measured rates to the offload planner
-(dkv_plan_offload), rebuilds the cache at the planned host fraction and
-reports the planned step: predicted against measured time and the HBM bytes
-the placement frees.
+--mode planned measures the workload at its own placement first (and, when
+the HBM budget allows, with the whole cache in HBM, for the HBM kernel's rate
+alone), gives the measured rates to the offload planner (dkv_plan_offload),
+rebuilds the cache at the planned host fraction and reports the planned step:
+predicted against measured time and the HBM bytes the placement frees.
 
 With N > 1 (launched by torchrun) every rank runs an independent replica of
 the workload on its own GPU and PCIe link; rank 0 prints the JSON line with
@@ -65,9 +65,14 @@ def parse_args(argv=None):
     ap.add_argument("--host-ctas", type=int, default=0)
     ap.add_argument("--ctx", type=int, default=0,
                     help="override the context length (a reduced case of the workload, e.g. for profiler captures)")
+    ap.add_argument("--host-fraction", type=float, default=-1.0,
+                    help="replace the workload's share of blocks in host memory (0..1; < 0: the workload's own)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    return ap.parse_args(argv)
+    args = ap.parse_args(argv)
+    if args.host_fraction > 1:
+        ap.error("--host-fraction must be at most 1")
+    return args
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -101,12 +106,15 @@ def barrier():
         dist.barrier()
 
 
-def workload_for_rank(name: str, rank: int, ctx: int = 0) -> kvgen.Workload:
+def workload_for_rank(name: str, rank: int, ctx: int = 0, host_fraction: float = -1.0) -> kvgen.Workload:
     """Replica r draws its own inputs: same shapes and recipe, seed + 1000 r.  ctx > 0 replaces the
-    context length (the workload is then named with a "_ctx<N>" suffix)."""
+    context length (the workload is then named with a "_ctx<N>" suffix); host_fraction >= 0 replaces the
+    share of blocks placed in host memory (suffix "_h<F>")."""
     w = kvgen.get(name)
     if ctx > 0:
         w = w.replace(name=f"{w.name}_ctx{ctx}", ctx=ctx)
+    if host_fraction >= 0:
+        w = w.replace(name=f"{w.name}_h{host_fraction:g}", host_fraction=host_fraction)
     return w if rank == 0 else w.replace(seed=w.seed + 1000 * rank)
 
 
@@ -249,7 +257,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    w = workload_for_rank(args.workload, 0, args.ctx)
+    w = workload_for_rank(args.workload, 0, args.ctx, args.host_fraction)
     lens = kvgen.gen_seq_lens(w)
     q = kvgen.gen_q(w)
     k, v = kvgen.gen_kv(w, lens)
@@ -383,7 +391,7 @@ def run_dkv(args):
     dist_init("nccl")
     import decode_attention_host_b200 as dkv
 
-    w = workload_for_rank(args.workload, rank, args.ctx)
+    w = workload_for_rank(args.workload, rank, args.ctx, args.host_fraction)
     q = kvgen.gen_q(w)
     lens = kvgen.gen_seq_lens(w)
     k, v = kvgen.gen_kv(w, lens)
@@ -437,7 +445,8 @@ def run_dkv(args):
     if planned:
         # The offload planner, fed with the two kernels' rates measured side by side.  Round 0 uses the rates
         # of the workload's own placement; each later round re-plans from the rates measured at the previous
-        # plan (the rates depend on the operating point), and stops once the fraction settles.
+        # plan (the rates depend on the operating point), and stops once the fraction settles.  The HBM
+        # kernel's rate alone comes from the all-HBM placement, measured once when the budget allows it.
         def rates_of(m):
             r = {k["kernel"]: k["achieved"] for k in m["kernels"] if "achieved" in k}
             return r.get("host_stream", b_pcie * 0.92), r.get("hbm_split_k", hbm_peak)
@@ -447,24 +456,42 @@ def run_dkv(args):
         rounds = [{"host_fraction": w.host_fraction, "measured_step_ms": meas["ms"], "host_stream_gbs": host_gbs,
                    "hbm_split_k_gbs": hbm_gbs}]
         f_prev = w.host_fraction
+        # When the budget lets the whole cache sit in HBM, the HBM kernel's rate alone (no host stream beside
+        # it) is measured too: the planner keeps everything in HBM if that is no slower.
+        alone_gbs, all_hbm_ms = -1.0, None
+        if (budget < 0 or budget >= x) and w.host_fraction > 0:
+            kv.free()
+            kv = paged(0.0)
+            meas = measure_placement(args, dkv, attn, kv, step, stream, device, b_pcie, hbm_peak, hbm_src, w.name,
+                                     args.mode)
+            alone_gbs, all_hbm_ms = rates_of(meas)[1], meas["ms"]
+            rounds.append({"host_fraction": 0.0, "measured_step_ms": all_hbm_ms, "hbm_split_k_gbs": alone_gbs})
+            f_prev = 0.0
         plan = None
         for _ in range(2):
-            plan = dkv.dkv_plan_offload(x, host_gbs, hbm_gbs, budget)
+            plan = dkv.dkv_plan_offload(x, host_gbs, hbm_gbs, budget, alone_gbs)
             if abs(plan.host_fraction - f_prev) < 1e-3:
+                if len(rounds) > 1 and "predicted_step_ms" not in rounds[-1]:
+                    rounds[-1].update({"rates_used_gbs": [host_gbs, hbm_gbs, alone_gbs],
+                                       "predicted_step_ms": plan.step_seconds * 1e3,
+                                       "predicted_over_measured": plan.step_seconds * 1e3 / meas["ms"]})
                 break
             kv.free()
             kv = paged(plan.host_fraction)
             meas = measure_placement(args, dkv, attn, kv, step, stream, device, b_pcie, hbm_peak, hbm_src, w.name,
                                      args.mode)
-            host_gbs, hbm_gbs = rates_of(meas)
-            rounds.append({"host_fraction": plan.host_fraction,
-                           "rates_used_gbs": [rounds[-1]["host_stream_gbs"], rounds[-1]["hbm_split_k_gbs"]],
+            used = [host_gbs, hbm_gbs, alone_gbs]
+            if plan.host_fraction > 0:   # the side-by-side rates of this placement feed the next round
+                host_gbs, hbm_gbs = rates_of(meas)
+            rounds.append({"host_fraction": plan.host_fraction, "rates_used_gbs": used,
                            "predicted_step_ms": plan.step_seconds * 1e3, "measured_step_ms": meas["ms"],
                            "predicted_over_measured": plan.step_seconds * 1e3 / meas["ms"],
-                           "host_stream_gbs": host_gbs, "hbm_split_k_gbs": hbm_gbs})
+                           "host_stream_gbs": rates_of(meas)[0] if plan.host_fraction > 0 else None,
+                           "hbm_split_k_gbs": rates_of(meas)[1]})
             f_prev = plan.host_fraction
         last = rounds[-1]
         planner = {"rounds": rounds, "hbm_budget_bytes": budget if budget >= 0 else None,
+                   "hbm_alone_gbs": alone_gbs if alone_gbs > 0 else None, "all_hbm_step_ms": all_hbm_ms,
                    "time_optimal_fraction": plan.time_optimal_fraction, "host_fraction": f_prev,
                    "predicted_step_ms": last.get("predicted_step_ms"), "measured_step_ms": meas["ms"],
                    "predicted_over_measured": last.get("predicted_over_measured"),

@@ -95,7 +95,7 @@ def _load() -> ctypes.CDLL:
         "dkv_plan_blocks": [c.POINTER(DkvPlanParams), vp, i32, vp, i32, c.POINTER(DkvPlanResult)],
         "dkv_pack_kv": [vp, vp, i64, vp, i32, i32, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp],
         "dkv_profile_begin": [vp, i32],
-        "dkv_plan_offload": [c.c_double, c.c_double, c.c_double, c.c_double, c.POINTER(DkvOffloadPlan)],
+        "dkv_plan_offload": [c.c_double, c.c_double, c.c_double, c.c_double, c.c_double, c.POINTER(DkvOffloadPlan)],
         "dkv_attn_decode_noalloc": [c.POINTER(DkvConfig), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32,
                                     i32],
         "dkv_profile_end": [vp, c.POINTER(c.c_float), c.POINTER(i32)],
@@ -211,11 +211,11 @@ def dkv_plan_blocks(params: DkvPlanParams, seq_lens: np.ndarray, block_table: np
     return res
 
 
-def dkv_plan_offload(kv_bytes: float, host_gbs: float, hbm_gbs: float, hbm_budget_bytes: float = -1.0
-                     ) -> DkvOffloadPlan:
+def dkv_plan_offload(kv_bytes: float, host_gbs: float, hbm_gbs: float, hbm_budget_bytes: float = -1.0,
+                     hbm_alone_gbs: float = -1.0) -> DkvOffloadPlan:
     plan = DkvOffloadPlan()
     _check(lib.dkv_plan_offload(float(kv_bytes), float(host_gbs), float(hbm_gbs), float(hbm_budget_bytes),
-                                ctypes.byref(plan)))
+                                float(hbm_alone_gbs), ctypes.byref(plan)))
     return plan
 
 

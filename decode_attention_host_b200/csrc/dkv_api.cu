@@ -83,16 +83,24 @@ constexpr int kDevTmaMode = DKV_DEV_TMA;
 #define DKV_HOST_TMA 0
 #endif
 constexpr bool kHostTma = DKV_HOST_TMA != 0;
-// Units per resident warp the single-token HBM kernel's split plan aims at
-// when that kernel has the GPU to itself (build-time knob, 1 to 4; the
-// partial-row workspace covers up to 4).  More, smaller units balance the
-// SMs better but add a query load, RoPE seeds and a partial write per unit;
-// 1 is the fastest measured.
-#ifndef DKV_DEV_OVERSUB
-#define DKV_DEV_OVERSUB 1
+// Units per resident warp of the single-token HBM kernel when it has the GPU
+// to itself and the batch holds 2 or more sequences (build-time knobs): up to
+// DKV_DEV_REFINE (1 to 8; the partial-row workspace covers 8) while each unit
+// keeps at least DKV_DEV_UNIT_TOKENS tokens.  With ragged lengths the plan,
+// sized by the table capacity, otherwise gives the longest sequences units as
+// long as a warp's whole share (an all-HBM batch of 16 sequences of 1k-16k
+// tokens ran 1.9x faster with 2 units per warp); uniform batches are
+// unchanged within 1%.  One sequence cannot be ragged and keeps one unit per
+// warp.
+#ifndef DKV_DEV_REFINE
+#define DKV_DEV_REFINE 2
 #endif
-constexpr int kDevOversub = DKV_DEV_OVERSUB;
-static_assert(kDevOversub >= 1 && kDevOversub <= 4, "DKV_DEV_OVERSUB must be 1..4");
+#ifndef DKV_DEV_UNIT_TOKENS
+#define DKV_DEV_UNIT_TOKENS 1024
+#endif
+constexpr int kDevRefine = DKV_DEV_REFINE;
+constexpr int kDevUnitTokens = DKV_DEV_UNIT_TOKENS;
+static_assert(kDevRefine >= 1 && kDevRefine <= 8, "DKV_DEV_REFINE must be 1..8");
 constexpr int kDefaultHostCtas = 16;
 constexpr int kListThreads = 1024;  // threads of the pool-lists kernel
 
@@ -270,6 +278,13 @@ void release(dkv_handle* h) {
 long launch_warps(const dkv_handle* h, bool beside_host) {
   const long ctas = 2L * h->sm_count - (beside_host ? static_cast<long>(h->host_ctas) * (2 - h->beside_host) : 0);
   return dkv::kWarps * (ctas > 1 ? ctas : 1);
+}
+
+// Split plan of the HBM kernel when it has the GPU to itself.
+dkv::SplitPlan alone_plan(const dkv_handle* h, int nblk, int batch, bool multi) {
+  const long per = static_cast<long>(batch) * h->cfg.num_kv_heads;
+  return dkv::plan_split_refined(nblk, per, h->cfg.block_size, launch_warps(h, false),
+                                 multi || batch < 2 ? 1 : kDevRefine, kDevUnitTokens);
 }
 
 // Whether one CTA of kernel b fits on an SM that holds one CTA of kernel a,
@@ -466,8 +481,7 @@ int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_table_strid
   if (batch < 0 || batch > h->cfg.max_batch || block_table_stride < 1)
     return fail(DKV_ERR_INVALID_ARG, "dkv_query_plan: batch or stride out of range");
   const int nblk = block_table_stride < h->cfg.max_blocks_per_seq ? block_table_stride : h->cfg.max_blocks_per_seq;
-  const dkv::SplitPlan pl =
-      dkv::plan_split(nblk, static_cast<long>(batch) * h->cfg.num_kv_heads, h->cfg.block_size, launch_warps(h, false), 0);
+  const dkv::SplitPlan pl = alone_plan(h, nblk, batch, false);
   *num_splits = pl.nsplit;
   *blocks_per_split = pl.bps;
   return DKV_OK;
@@ -546,8 +560,8 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   const long per = static_cast<long>(batch) * c.num_kv_heads;
   const long host_warps = staged ? launch_warps(h, false) : static_cast<long>(dkv::kWarps) * h->host_ctas;
   const dkv::SplitPlan ph = dkv::plan_split(nblk_cap, per, c.block_size, host_warps, 0);
-  const dkv::SplitPlan pd =
-      dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, concurrent) * (concurrent || multi ? 1 : kDevOversub), 0);
+  const dkv::SplitPlan pd = concurrent ? dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, true), 0)
+                                        : alone_plan(h, nblk_cap, batch, multi);
   const int nsplit_h = run_host ? ph.nsplit : 0;
   const int nsplit_d = run_dev ? pd.nsplit : 0;
   const int nslots = nsplit_h + nsplit_d;

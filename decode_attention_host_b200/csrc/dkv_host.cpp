@@ -120,23 +120,34 @@ int dkv_plan_blocks(const dkv_plan_params* params, const int32_t* seq_lens, int3
   return DKV_OK;
 }
 
-int dkv_plan_offload(double kv_bytes, double host_gbs, double hbm_gbs, double hbm_budget_bytes,
+int dkv_plan_offload(double kv_bytes, double host_gbs, double hbm_gbs, double hbm_budget_bytes, double hbm_alone_gbs,
                      dkv_offload_plan* plan) {
   if (!plan || !(kv_bytes > 0.0) || !(host_gbs > 0.0) || !(hbm_gbs > 0.0) || std::isnan(hbm_budget_bytes) ||
-      !std::isfinite(kv_bytes) || !std::isfinite(host_gbs) || !std::isfinite(hbm_gbs))
+      !std::isfinite(kv_bytes) || !std::isfinite(host_gbs) || !std::isfinite(hbm_gbs) ||
+      !std::isfinite(hbm_alone_gbs))
     return set_error(DKV_ERR_INVALID_ARG, "dkv_plan_offload: sizes and bandwidths must be positive and finite");
-  const double f_time = host_gbs / (host_gbs + hbm_gbs);
+  // best split with both kernels running: the two sides finish together
+  const double f_conc = host_gbs / (host_gbs + hbm_gbs);
+  const double t_conc = kv_bytes / ((host_gbs + hbm_gbs) * 1e9);
+  // everything in HBM, the HBM kernel alone, when that is no slower
+  const bool alone_wins = hbm_alone_gbs > 0.0 && kv_bytes / (hbm_alone_gbs * 1e9) <= t_conc;
   double f_cap = 0.0;
   if (hbm_budget_bytes >= 0.0) f_cap = 1.0 - hbm_budget_bytes / kv_bytes;
-  double f = f_time > f_cap ? f_time : f_cap;
-  if (f > 1.0) f = 1.0;
-  if (f < 0.0) f = 0.0;
-  const double t_host = f * kv_bytes / (host_gbs * 1e9);
-  const double t_dev = (1.0 - f) * kv_bytes / (hbm_gbs * 1e9);
+  double f, t;
+  if (alone_wins && f_cap <= 0.0) {
+    f = 0.0;
+    t = kv_bytes / (hbm_alone_gbs * 1e9);
+  } else {
+    f = f_conc > f_cap ? f_conc : f_cap;
+    if (f > 1.0) f = 1.0;
+    const double t_host = f * kv_bytes / (host_gbs * 1e9);
+    const double t_dev = (1.0 - f) * kv_bytes / (hbm_gbs * 1e9);
+    t = t_host > t_dev ? t_host : t_dev;
+  }
   plan->host_fraction = f;
-  plan->step_seconds = t_host > t_dev ? t_host : t_dev;
+  plan->step_seconds = t;
   plan->hbm_bytes_freed = f * kv_bytes;
-  plan->time_optimal_fraction = f_time;
+  plan->time_optimal_fraction = alone_wins ? 0.0 : f_conc;
   return DKV_OK;
 }
 

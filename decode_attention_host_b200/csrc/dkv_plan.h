@@ -42,6 +42,24 @@ inline SplitPlan plan_split(int nblk, long per, int block_size, long warps, long
   return r;
 }
 
+// Finer splits for long units.  Units are handed out dynamically, so a batch
+// of ragged lengths finishes when its longest unit does, and a plan sized by
+// the table capacity makes the units of the longest sequences as long as a
+// warp's whole share.  This plans for `factor` units per resident warp (a
+// whole number per warp, so that no second round of units runs on part of
+// the warps), stepping the factor down until each unit keeps at least
+// `min_tokens` tokens, so that a unit's setup (query load, RoPE seeds,
+// partial write) stays small against its tiles.  Never gives fewer splits
+// than the plan for one unit per warp.
+inline SplitPlan plan_split_refined(int nblk, long per, int block_size, long warps, int factor, int min_tokens) {
+  const SplitPlan base = plan_split(nblk, per, block_size, warps, 0);
+  for (int k = factor; k > 1; --k) {
+    const SplitPlan r = plan_split(nblk, per, block_size, warps * k, 0);
+    if (static_cast<long>(r.bps) * block_size >= min_tokens && r.nsplit > base.nsplit) return r;
+  }
+  return base;
+}
+
 // The minimum split size in blocks: the blocks-per-split floor of every plan.
 inline int min_blocks_per_split(int block_size) {
   const int m = (kMinSplitTokens + block_size - 1) / block_size;

@@ -209,11 +209,13 @@ DKV_API int dkv_last_launch_count(const dkv_handle* h, int32_t* count);
 
 /* dkv_query_plan -- the split-K decomposition of the HBM kernel of a
  * dkv_attn_decode call whose blocks all sit in HBM, for (batch,
- * block_table_stride): splits per sequence and blocks per split.  The splits
- * never make more units (batch * splits * Hkv) than the kernel's resident
- * warps.  With host blocks as well, each launch splits the list of its own
- * pool's blocks of every sequence, and the HBM launch plans for the warps
- * left beside the zero-copy host kernel. */
+ * block_table_stride): splits per sequence and blocks per split.  The plan
+ * aims at one unit (sequence, split, kv head) per resident warp of the
+ * kernel; with 2 or more sequences, at 2 units per warp when every unit still
+ * holds at least 1024 tokens (finer units keep ragged batches balanced).
+ * With host blocks as well, each launch splits the list of its own pool's
+ * blocks of every sequence, and the HBM launch plans one unit per warp left
+ * beside the zero-copy host kernel. */
 DKV_API int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_table_stride, int32_t* num_splits,
                    int32_t* blocks_per_split);
 
@@ -376,18 +378,26 @@ DKV_API int dkv_plan_blocks(const dkv_plan_params* params, const int32_t* seq_le
  * README, Key Features: placement / offloading-ratio utilities; DirectKV
  * README, Figure mapping, Fig 11b: GPU memory freed at long context).
  * With X = total KV bytes, the modelled step time of a placement with host
- * fraction f is T(f) = max(f*X / host_gbs, (1-f)*X / hbm_gbs): the zero-copy
- * host stream and the HBM kernel run concurrently and the slower one sets the
- * step.  T falls while the HBM side dominates and rises once PCIe does, so the
- * time-optimal fraction is f* = host_gbs / (host_gbs + hbm_gbs).  An HBM budget
- * for the cache forces f >= 1 - budget/X.  The plan is f = max(f*, that bound),
- * capped at 1.
+ * fraction f > 0 is T(f) = max(f*X / host_gbs, (1-f)*X / hbm_gbs): the
+ * zero-copy host stream and the HBM kernel run concurrently and the slower one
+ * sets the step.  T falls while the HBM side dominates and rises once PCIe
+ * does, so the best such fraction is f* = host_gbs / (host_gbs + hbm_gbs),
+ * with T(f*) = X / (host_gbs + hbm_gbs).  At f = 0 the HBM kernel runs alone,
+ * T(0) = X / hbm_alone_gbs, which can be shorter: a kernel beside the host
+ * stream is slower than alone.  An HBM budget for the cache forces
+ * f >= 1 - budget/X.  The plan is f = 0 when the budget allows it and
+ * T(0) <= T(f*); otherwise f = max(f*, that bound), capped at 1.
  *   kv_bytes        X > 0
- *   host_gbs        measured host read bandwidth the kernel achieves (> 0)
- *   hbm_gbs         measured HBM read bandwidth (> 0)
+ *   host_gbs        measured host read bandwidth of the host kernel (> 0)
+ *   hbm_gbs         measured HBM read bandwidth of the HBM kernel while the
+ *                   host kernel runs beside it (> 0)
  *   hbm_budget_bytes  HBM bytes the cache may occupy; < 0 means unlimited
+ *   hbm_alone_gbs   measured HBM read bandwidth of the HBM kernel alone;
+ *                   <= 0 if unknown (then f = 0 is never chosen)
  * Out: host_fraction, predicted step seconds, HBM bytes freed (f*X) and the
- * time-optimal fraction f*.  Pure host arithmetic; errors: INVALID_ARG. */
+ * time-optimal fraction without a budget (0 or f*).  Pure host arithmetic;
+ * errors: INVALID_ARG (sizes or rates not positive and finite, a NaN budget,
+ * a non-finite hbm_alone_gbs). */
 typedef struct dkv_offload_plan {
   double host_fraction;
   double step_seconds;
@@ -396,7 +406,7 @@ typedef struct dkv_offload_plan {
 } dkv_offload_plan;
 
 DKV_API int dkv_plan_offload(double kv_bytes, double host_gbs, double hbm_gbs, double hbm_budget_bytes,
-                             dkv_offload_plan* plan);
+                             double hbm_alone_gbs, dkv_offload_plan* plan);
 
 /*
  * dkv_pack_kv -- write logical K/V into the paged pools following a table.

@@ -81,3 +81,13 @@ def test_default_workload_is_the_largest_single_gpu_config():
     import kvgen
     sizes = {n: kvgen.get(n).batch * kvgen.get(n).max_ctx for n in ("tiny_gqa", "llama3_8b", "long_ctx", "opt_6_7b")}
     assert max(sizes, key=sizes.get) == "long_ctx"
+
+
+def test_host_fraction_override_names_the_placement():
+    import bench
+    w = bench.workload_for_rank("opt_6_7b", 0, 0, 0.0)
+    assert w.host_fraction == 0.0 and w.name == "opt_6_7b_h0"
+    assert bench.workload_for_rank("opt_6_7b", 0).host_fraction == 0.75
+    assert bench.workload_for_rank("long_ctx", 1, 4096, 0.5).name == "long_ctx_ctx4096_h0.5"
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--host-fraction", "1.5"])

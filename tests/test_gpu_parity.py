@@ -201,6 +201,31 @@ def test_full_size_sampled_against_oracle(name, groups):
     case.free()
 
 
+@pytest.mark.parametrize("name,groups", [("opt_6_7b", 6), ("llama3_8b", 6), ("long_ctx", 3)])
+def test_full_size_all_in_hbm_sampled_against_oracle(name, groups):
+    """The named workloads with every block in HBM: the HBM kernel alone, with the plan of two units per warp
+    when the batch holds several sequences (opt_6_7b: 16 sequences of 1k-16k tokens, 4 splits of 256
+    blocks) and one per warp for a single sequence (long_ctx).  Sampled groups against the oracle."""
+    w = kvgen.get(name).replace(host_fraction=0.0)
+    case = gc.Case(w)
+    got = case.run()
+    assert np.isfinite(got).all()
+    assert case.attn.status() == 0 and case.kv.host_split == 0 and case.attn.launches() == 2
+    if name == "opt_6_7b":
+        # 1024 table blocks per sequence, 16 x 32 (sequence, kv head) pairs; one unit per warp of 2 CTAs x 4
+        # warps per SM would give floor(8 SMs / 512) splits, two units per warp twice that
+        warps = 8 * torch.cuda.get_device_properties(0).multi_processor_count
+        one = max(1, warps // 512)
+        nsplit, bps = case.attn.plan(w.batch, case.kv.stride)
+        assert nsplit == -(-1024 // -(-1024 // (2 * one))) and bps * 16 >= 1024
+    mask = gc.sampled_groups(w, groups, 321)
+    err = gc.sampled_err(w, got, case.oracle(group_mask=mask), mask)
+    gc.record("test_full_size_all_in_hbm_sampled_against_oracle", name + "_h0", err,
+              f"{int(mask.sum())} of {mask.size}")
+    assert err <= gc.TOL, f"{name}: {err:.3e}"
+    case.free()
+
+
 @pytest.mark.parametrize("cell", [c.name for c in kvgen.sweep_cells()])
 def test_every_sweep_cell_full_size_sampled(cell):
     """All 20 context x host-fraction cells at full size (B=4, 1% outlier keys x8), in the bench's launch

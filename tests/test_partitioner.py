@@ -157,8 +157,58 @@ def test_offload_step_time_is_minimal_at_the_plan():
         assert t >= plan.step_seconds - 1e-15
 
 
+def test_offload_all_hbm_when_the_kernel_alone_beats_the_concurrent_split():
+    """At f = 0 the HBM kernel has the GPU to itself; when its alone rate is at least the two sides' concurrent
+    rates together, keeping the whole cache in HBM is the fastest placement the budget allows."""
+    X, hb, beside, alone = 4 * (1 << 30), 51.3, 4570.0, 5580.0
+    plan = dkv.dkv_plan_offload(X, hb, beside, hbm_alone_gbs=alone)
+    assert plan.host_fraction == 0.0 and plan.time_optimal_fraction == 0.0 and plan.hbm_bytes_freed == 0.0
+    assert abs(plan.step_seconds - X / (alone * 1e9)) < 1e-15
+    # an unlimited budget (< 0) and a budget of the whole cache both allow it
+    assert dkv.dkv_plan_offload(X, hb, beside, float(X), alone).host_fraction == 0.0
+    # a budget below the cache forces a concurrent split, planned from the side-by-side rates alone
+    capped = dkv.dkv_plan_offload(X, hb, beside, 0.5 * X, alone)
+    assert abs(capped.host_fraction - 0.5) < 1e-12 and capped.time_optimal_fraction == 0.0
+    assert abs(capped.step_seconds - 0.5 * X / (hb * 1e9)) < 1e-12
+    small = dkv.dkv_plan_offload(X, hb, beside, 0.999 * X, alone)   # the bound is below f*: the concurrent optimum
+    assert abs(small.host_fraction - hb / (hb + beside)) < 1e-15
+
+
+def test_offload_keeps_the_concurrent_split_when_it_is_faster():
+    X, hb, beside = 1 << 30, 51.5, 6547.8
+    f = hb / (hb + beside)
+    for alone in (-1.0, 0.0, 6000.0, hb + beside - 1e-6):   # unknown, or slower than both sides together
+        plan = dkv.dkv_plan_offload(X, hb, beside, hbm_alone_gbs=alone)
+        assert abs(plan.host_fraction - f) < 1e-15 and abs(plan.time_optimal_fraction - f) < 1e-15
+        assert abs(plan.step_seconds - X / ((hb + beside) * 1e9)) < 1e-15
+    tie = dkv.dkv_plan_offload(X, hb, beside, hbm_alone_gbs=hb + beside)   # equal times: no host traffic
+    assert tie.host_fraction == 0.0
+
+
+@pytest.mark.parametrize("alone", [3000.0, 6000.0, 7000.0, 9000.0])
+@pytest.mark.parametrize("budget_frac", [-1.0, 1.0, 0.7, 0.2])
+def test_offload_plan_is_minimal_over_the_placements_the_budget_allows(alone, budget_frac):
+    """Brute force over f on a fine grid, with T(0) = X / alone and T(f > 0) = max(f X / hb, (1 - f) X / hbm)."""
+    X, hb, beside = 1e9, 50.0, 6500.0
+    budget = budget_frac * X if budget_frac >= 0 else -1.0
+    plan = dkv.dkv_plan_offload(X, hb, beside, budget, alone)
+    f_min = 0.0 if budget < 0 else max(0.0, 1.0 - budget / X)
+    best = None
+    for f in np.concatenate([[0.0], np.linspace(1e-6, 1.0, 200001)]):
+        if f < f_min - 1e-12:
+            continue
+        t = X / (alone * 1e9) if f == 0.0 else max(f * X / (hb * 1e9), (1 - f) * X / (beside * 1e9))
+        best = t if best is None else min(best, t)
+    assert plan.step_seconds <= best * (1 + 1e-9)
+    assert plan.host_fraction >= f_min - 1e-12
+    t_plan = X / (alone * 1e9) if plan.host_fraction == 0.0 else max(
+        plan.host_fraction * X / (hb * 1e9), (1 - plan.host_fraction) * X / (beside * 1e9))
+    assert abs(t_plan - plan.step_seconds) < 1e-15
+
+
 @pytest.mark.parametrize("args", [(0, 50, 7000, -1), (1e9, 0, 7000, -1), (1e9, 50, -1, -1), (float("inf"), 50, 7000, -1),
-                                  (1e9, 50, 7000, float("nan"))])
+                                  (1e9, 50, 7000, float("nan")), (1e9, 50, 7000, -1, float("nan")),
+                                  (1e9, 50, 7000, -1, float("inf"))])
 def test_offload_rejects_bad_inputs(args):
     with pytest.raises(dkv.DkvError):
         dkv.dkv_plan_offload(*args)

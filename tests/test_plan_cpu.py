@@ -4,7 +4,9 @@ Both live in the host-only header dkv_plan.h.  A small C++ program compiled with
 g++ sweeps the arguments the library can pass and checks, for every plan:
 1 <= nsplit <= max(1, warps / (batch * kv heads)), nsplit within the cap when
 one is given, nsplit * bps covering the blocks with no empty last split, and
-bps at least the minimum split size.  For the scratch bound it checks that the
+bps at least the minimum split size; for the refined plan (several units per
+warp), no fewer splits than one unit per warp, at most `factor` units per
+warp, and units of at least the minimum tokens whenever it refines.  For the scratch bound it checks that the
 returned number of slots fits the fixed array and one more does not.
 """
 import shutil
@@ -46,6 +48,39 @@ int main() {
       }
     }
   }
+  // the refined plan: never fewer splits than one unit per warp; when it
+  // refines, units of at least min_tokens and at most factor units per warp
+  long refined = 0;
+  for (int nblk = 1; nblk <= 70000; nblk += (nblk < 300 ? 7 : 1997)) {
+    for (long per : {8L, 32L, 512L}) {
+      for (int bs : {16, 32, 64}) {
+        for (long warps : {1184L, 4096L}) {
+          for (int factor : {1, 2, 4}) {
+            for (int min_tokens : {64, 1024}) {
+              const dkv::SplitPlan base = dkv::plan_split(nblk, per, bs, warps, 0);
+              const dkv::SplitPlan r = dkv::plan_split_refined(nblk, per, bs, warps, factor, min_tokens);
+              long target = factor * warps / per;
+              if (target < 1) target = 1;
+              ++plans;
+              bad += r.nsplit < base.nsplit;
+              bad += static_cast<long>(r.nsplit) * r.bps < nblk;
+              bad += static_cast<long>(r.nsplit - 1) * r.bps >= nblk;
+              bad += r.bps < dkv::min_blocks_per_split(bs);
+              bad += r.nsplit > target;
+              if (r.nsplit != base.nsplit) {
+                ++refined;
+                bad += factor == 1;
+                bad += static_cast<long>(r.bps) * bs < min_tokens;
+              } else {
+                bad += r.bps != base.bps;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+  bad += refined == 0;
   const size_t scratch = 16u << 20;
   for (size_t batch : {1ul, 2ul, 5ul, 8ul, 64ul, 300ul, 4000ul, 5000ul}) {
     for (size_t nblk : {0ul, 1ul, 2048ul, 16384ul, 100000ul}) {
