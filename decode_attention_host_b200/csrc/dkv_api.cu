@@ -83,14 +83,15 @@ constexpr int kDevTmaMode = DKV_DEV_TMA;
 #define DKV_HOST_TMA 0
 #endif
 constexpr bool kHostTma = DKV_HOST_TMA != 0;
-// Units per resident warp of the single-token HBM kernel when it has the GPU
-// to itself and the batch holds 2 or more sequences (build-time knobs): up to
+// Units per resident warp of the HBM kernel (single- or multi-token) when all
+// blocks sit in HBM and the batch holds 2 or more sequences (build-time
+// knobs): up to
 // DKV_DEV_REFINE (1 to 8; the partial-row workspace covers 8) while each unit
 // keeps at least DKV_DEV_UNIT_TOKENS tokens.  With ragged lengths the plan,
 // sized by the table capacity, otherwise gives the longest sequences units as
 // long as a warp's whole share (an all-HBM batch of 16 sequences of 1k-16k
-// tokens ran 1.9x faster with 2 units per warp); uniform batches are
-// unchanged within 1%.  One sequence cannot be ragged and keeps one unit per
+// tokens ran 1.9x faster with 2 units per warp, with 4 query tokens 1.95x);
+// uniform batches are unchanged within 1%.  One sequence cannot be ragged and keeps one unit per
 // warp.
 #ifndef DKV_DEV_REFINE
 #define DKV_DEV_REFINE 2
@@ -280,11 +281,12 @@ long launch_warps(const dkv_handle* h, bool beside_host) {
   return dkv::kWarps * (ctas > 1 ? ctas : 1);
 }
 
-// Split plan of the HBM kernel when it has the GPU to itself.
-dkv::SplitPlan alone_plan(const dkv_handle* h, int nblk, int batch, bool multi) {
+// Split plan of the HBM kernel of a call whose blocks all sit in HBM (the
+// only split launch of the call).
+dkv::SplitPlan alone_plan(const dkv_handle* h, int nblk, int batch) {
   const long per = static_cast<long>(batch) * h->cfg.num_kv_heads;
   return dkv::plan_split_refined(nblk, per, h->cfg.block_size, launch_warps(h, false),
-                                 multi || batch < 2 ? 1 : kDevRefine, kDevUnitTokens);
+                                 batch < 2 ? 1 : kDevRefine, kDevUnitTokens);
 }
 
 // Whether one CTA of kernel b fits on an SM that holds one CTA of kernel a,
@@ -481,7 +483,7 @@ int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_table_strid
   if (batch < 0 || batch > h->cfg.max_batch || block_table_stride < 1)
     return fail(DKV_ERR_INVALID_ARG, "dkv_query_plan: batch or stride out of range");
   const int nblk = block_table_stride < h->cfg.max_blocks_per_seq ? block_table_stride : h->cfg.max_blocks_per_seq;
-  const dkv::SplitPlan pl = alone_plan(h, nblk, batch, false);
+  const dkv::SplitPlan pl = alone_plan(h, nblk, batch);
   *num_splits = pl.nsplit;
   *blocks_per_split = pl.bps;
   return DKV_OK;
@@ -560,8 +562,8 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   const long per = static_cast<long>(batch) * c.num_kv_heads;
   const long host_warps = staged ? launch_warps(h, false) : static_cast<long>(dkv::kWarps) * h->host_ctas;
   const dkv::SplitPlan ph = dkv::plan_split(nblk_cap, per, c.block_size, host_warps, 0);
-  const dkv::SplitPlan pd = concurrent ? dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, true), 0)
-                                        : alone_plan(h, nblk_cap, batch, multi);
+  const dkv::SplitPlan pd = run_host ? dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, concurrent), 0)
+                                      : alone_plan(h, nblk_cap, batch);
   const int nsplit_h = run_host ? ph.nsplit : 0;
   const int nsplit_d = run_dev ? pd.nsplit : 0;
   const int nslots = nsplit_h + nsplit_d;

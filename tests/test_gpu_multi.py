@@ -16,9 +16,9 @@ from tests import gpu_cases as gc
 pytestmark = pytest.mark.gpu
 
 
-def _run(w: kvgen.Workload, tq: int, seed: int, lens=None):
+def _run(w: kvgen.Workload, tq: int, seed: int, lens=None, stride=None):
     lens = kvgen.gen_seq_lens(w) if lens is None else np.asarray(lens, dtype=np.int32)
-    case = gc.Case(w, lens=lens + tq - 1, max_batch=w.batch * tq)
+    case = gc.Case(w, lens=lens + tq - 1, max_batch=w.batch * tq, stride=stride)
     q = np.random.default_rng(seed).standard_normal((w.batch, tq, w.num_q_heads, w.head_dim)).astype(np.float32)
     case.kv.seq_lens_dev.copy_(torch.from_numpy(lens))
     out = torch.full((w.batch, tq, w.num_q_heads, w.head_dim), float("nan"), device="cuda")
@@ -50,6 +50,22 @@ def test_mha_chunk_queries_fp16(tq):
     w = kvgen.OPT_6_7B.replace(name=f"multi_mha_{tq}", batch=2, num_q_heads=4, num_kv_heads=4, ctx=(50, 700),
                                seed=80 + tq)
     case, lens, q, got = _run(w, tq, 90 + tq)
+    _check(case, lens, q, got)
+    case.free()
+
+
+def test_all_in_hbm_with_two_units_per_warp():
+    """Every block in HBM and a table capacity of 4736 blocks of 16 tokens: the plan takes two units per warp
+    of at least 1024 tokens (twice the splits of one unit per warp), so with sequences of 100-3000 tokens most
+    units are empty and the rest hold the sequences' first blocks."""
+    w = kvgen.LLAMA3_8B.replace(name="multi_refined", batch=4, ctx=(100, 3000), host_fraction=0.0, seed=97)
+    case, lens, q, got = _run(w, 4, 98, stride=4736)
+    warps = 8 * torch.cuda.get_device_properties(0).multi_processor_count
+    per = w.batch * w.num_kv_heads
+    one = -(-4736 // -(-4736 // max(1, warps // per)))
+    nsplit, bps = case.attn.plan(w.batch, case.kv.stride)
+    assert nsplit > one and bps * w.block_size >= 1024 and nsplit * bps >= 4736
+    assert case.kv.host_split == 0 and case.attn.launches() == 2
     _check(case, lens, q, got)
     case.free()
 
