@@ -175,7 +175,7 @@ SplitEntry pick_multi(int D, bool bf16, bool rope) {
 }
 
 // shared memory of the multi-token kernel: per warp a 2-stage (K, V) ring and one rotated-K lo tile
-size_t multi_smem(int D) { return static_cast<size_t>(dkv::kWarps) * 5 * dkv::kTileTokens * D * 2; }
+size_t multi_smem(int D) { return dkv::multi_smem_bytes(D); }
 
 // The merge, optionally as a programmatic dependent launch of the split kernel
 // just before it on the stream: its grid is set up while that kernel drains

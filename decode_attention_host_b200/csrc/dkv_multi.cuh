@@ -24,10 +24,20 @@
 namespace dkv {
 
 constexpr int kMultiMaxRows = 16;
+#ifndef DKV_MULTI_STAGES
+#define DKV_MULTI_STAGES 2
+#endif
+constexpr int kMultiStages = DKV_MULTI_STAGES;  // ring depth of the multi-token kernel (build-time knob)
+
+// Dynamic shared memory of multi_kernel<D, *, *>: per warp the K and V tiles
+// of every ring stage plus the lo tile of the rotated K.
+__host__ __device__ constexpr size_t multi_smem_bytes(int D) {
+  return static_cast<size_t>(kWarps) * (2 * kMultiStages + 1) * kTileTokens * D * 2;
+}
 
 template <int D, bool BF16, bool ROPE>
 __global__ void __launch_bounds__(kThreads) multi_kernel(const SplitParams p) {
-  constexpr int NST = 2;                       // ring depth (one tile in flight)
+  constexpr int NST = kMultiStages;            // ring depth (NST - 1 tiles in flight)
   constexpr int PPL = D / 16;                  // NeoX pairs per lane in the rotation pass
   constexpr int NP2 = PPL / 2;
   constexpr int ROW = D * 2;
