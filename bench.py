@@ -443,9 +443,9 @@ def run_dkv(args):
                              args.mode)
     planner = None
     if planned:
-        # The offload planner, fed with the two kernels' rates measured side by side.  Round 0 uses the rates
-        # of the workload's own placement; each later round re-plans from the rates measured at the previous
-        # plan (the rates depend on the operating point), and stops once the fraction settles.  The HBM
+        # The offload planner, fed with the two kernels' rates measured side by side.  The first plan uses the
+        # rates of the workload's own placement; each later plan uses the rates measured at the previous plan
+        # (the rates depend on the operating point), until the fraction settles.  The HBM
         # kernel's rate alone comes from the all-HBM placement, measured once when the budget allows it.
         def rates_of(m):
             r = {k["kernel"]: k["achieved"] for k in m["kernels"] if "achieved" in k}
