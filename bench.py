@@ -252,6 +252,18 @@ def oracle_gbs(w: kvgen.Workload, q, k, v, lens, group_mask, min_seconds: float 
 
 # ----------------------------------------------------------------------------- reference arm (the oracle)
 
+def cpu_model() -> str:
+    """The host CPU's model name, as the kernel reports it."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -282,7 +294,7 @@ def run_reference(args):
         "ms_per_step": 1e3 * total_bytes / (value * 1e9), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args.gpus),
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "cpu": cpu_model(),
                          "sample": f"{per_step} of {ngroups} (batch, kv head) groups per step; ms_per_step "
                                    f"extrapolates to the whole batch"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -557,7 +569,7 @@ def run_dkv(args):
         ngroups = w.batch * w.num_kv_heads
         mask = np.ones((w.batch, w.num_kv_heads), dtype=np.uint8)
         gbs, sec, threads, reps = oracle_gbs(w, q, k, v, lens, mask)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "cpu": cpu_model(),
                "sample": f"all {ngroups} (batch, kv head) groups of one step, run {reps} times: {sec:.1f} s"}
 
     if e2e is not None:
