@@ -252,6 +252,61 @@ def oracle_gbs(w: kvgen.Workload, q, k, v, lens, group_mask, min_seconds: float 
 
 # ----------------------------------------------------------------------------- reference arm (the oracle)
 
+def plan_placement(plan_offload, measure_at, rates_of, x: float, budget: float, f0: float, meas0: dict):
+    """The offload-planner rounds of --mode planned.
+
+    plan_offload is dkv_plan_offload; measure_at(f) rebuilds the cache with host fraction f and measures a step
+    there (a dict with "ms"); rates_of(m) gives the host-stream and HBM kernels' GB/s measured in m.  Rounds:
+    the workload's own placement f0 (meas0); when the budget lets the whole cache sit in HBM, that placement,
+    for the HBM kernel's rate alone; the side-by-side split, re-planned from the rates measured at the previous
+    split (they depend on the operating point) until it settles; finally the plan that weighs that split
+    against the whole cache in HBM, measured there unless the last round already was.  Returns the planner
+    record and the measurement of the chosen placement, whose cache measure_at left built."""
+    host_gbs, hbm_gbs = rates_of(meas0)
+    rounds = [{"host_fraction": f0, "measured_step_ms": meas0["ms"], "host_stream_gbs": host_gbs,
+               "hbm_split_k_gbs": hbm_gbs}]
+    meas, f_cur = meas0, f0
+    alone_gbs, all_hbm_ms = -1.0, None
+    if f0 == 0:   # the workload's own placement is the whole cache in HBM
+        alone_gbs, all_hbm_ms = hbm_gbs, meas0["ms"]
+    elif budget < 0 or budget >= x:
+        meas, f_cur = measure_at(0.0), 0.0
+        alone_gbs, all_hbm_ms = rates_of(meas)[1], meas["ms"]
+        rounds.append({"host_fraction": 0.0, "measured_step_ms": all_hbm_ms, "hbm_split_k_gbs": alone_gbs})
+    split_fs = [f0] if f0 > 0 else []
+
+    def measure_round(plan, used):
+        m = measure_at(plan.host_fraction)
+        h, d = rates_of(m)
+        rounds.append({"host_fraction": plan.host_fraction, "rates_used_gbs": used,
+                       "predicted_step_ms": plan.step_seconds * 1e3, "measured_step_ms": m["ms"],
+                       "predicted_over_measured": plan.step_seconds * 1e3 / m["ms"],
+                       "host_stream_gbs": h if plan.host_fraction > 0 else None, "hbm_split_k_gbs": d})
+        return m
+
+    for _ in range(2):
+        split = plan_offload(x, host_gbs, hbm_gbs, budget, -1.0)   # the side-by-side split alone
+        if any(abs(split.host_fraction - f) < 1e-3 for f in split_fs):
+            break
+        meas, f_cur = measure_round(split, [host_gbs, hbm_gbs, -1.0]), split.host_fraction
+        split_fs.append(f_cur)
+        host_gbs, hbm_gbs = rates_of(meas)
+    plan = plan_offload(x, host_gbs, hbm_gbs, budget, alone_gbs)
+    if abs(plan.host_fraction - f_cur) >= 1e-3:
+        meas, f_cur = measure_round(plan, [host_gbs, hbm_gbs, alone_gbs]), plan.host_fraction
+    elif "predicted_step_ms" not in rounds[-1]:
+        rounds[-1].update({"rates_used_gbs": [host_gbs, hbm_gbs, alone_gbs],
+                           "predicted_step_ms": plan.step_seconds * 1e3,
+                           "predicted_over_measured": plan.step_seconds * 1e3 / meas["ms"]})
+    last = rounds[-1]
+    planner = {"rounds": rounds, "hbm_budget_bytes": budget if budget >= 0 else None,
+               "hbm_alone_gbs": alone_gbs if alone_gbs > 0 else None, "all_hbm_step_ms": all_hbm_ms,
+               "time_optimal_fraction": plan.time_optimal_fraction, "host_fraction": f_cur,
+               "predicted_step_ms": last.get("predicted_step_ms"), "measured_step_ms": meas["ms"],
+               "predicted_over_measured": last.get("predicted_over_measured")}
+    return planner, meas
+
+
 def cpu_model() -> str:
     """The host CPU's model name, as the kernel reports it."""
     try:
@@ -455,60 +510,21 @@ def run_dkv(args):
                              args.mode)
     planner = None
     if planned:
-        # The offload planner, fed with the two kernels' rates measured side by side.  The first plan uses the
-        # rates of the workload's own placement; each later plan uses the rates measured at the previous plan
-        # (the rates depend on the operating point), until the fraction settles.  The HBM
-        # kernel's rate alone comes from the all-HBM placement, measured once when the budget allows it.
         def rates_of(m):
             r = {k["kernel"]: k["achieved"] for k in m["kernels"] if "achieved" in k}
             return r.get("host_stream", b_pcie * 0.92), r.get("hbm_split_k", hbm_peak)
+
+        def measure_at(f):
+            nonlocal kv
+            kv.free()
+            kv = paged(f)
+            return measure_placement(args, dkv, attn, kv, step, stream, device, b_pcie, hbm_peak, hbm_src, w.name,
+                                     args.mode)
         x = float(meas["kv_bytes"])
         budget = args.hbm_budget_frac * x if args.hbm_budget_frac >= 0 else -1.0
-        host_gbs, hbm_gbs = rates_of(meas)
-        rounds = [{"host_fraction": w.host_fraction, "measured_step_ms": meas["ms"], "host_stream_gbs": host_gbs,
-                   "hbm_split_k_gbs": hbm_gbs}]
-        f_prev = w.host_fraction
-        # When the budget lets the whole cache sit in HBM, the HBM kernel's rate alone (no host stream beside
-        # it) is measured too: the planner keeps everything in HBM if that is no slower.
-        alone_gbs, all_hbm_ms = -1.0, None
-        if (budget < 0 or budget >= x) and w.host_fraction > 0:
-            kv.free()
-            kv = paged(0.0)
-            meas = measure_placement(args, dkv, attn, kv, step, stream, device, b_pcie, hbm_peak, hbm_src, w.name,
-                                     args.mode)
-            alone_gbs, all_hbm_ms = rates_of(meas)[1], meas["ms"]
-            rounds.append({"host_fraction": 0.0, "measured_step_ms": all_hbm_ms, "hbm_split_k_gbs": alone_gbs})
-            f_prev = 0.0
-        plan = None
-        for _ in range(2):
-            plan = dkv.dkv_plan_offload(x, host_gbs, hbm_gbs, budget, alone_gbs)
-            if abs(plan.host_fraction - f_prev) < 1e-3:
-                if len(rounds) > 1 and "predicted_step_ms" not in rounds[-1]:
-                    rounds[-1].update({"rates_used_gbs": [host_gbs, hbm_gbs, alone_gbs],
-                                       "predicted_step_ms": plan.step_seconds * 1e3,
-                                       "predicted_over_measured": plan.step_seconds * 1e3 / meas["ms"]})
-                break
-            kv.free()
-            kv = paged(plan.host_fraction)
-            meas = measure_placement(args, dkv, attn, kv, step, stream, device, b_pcie, hbm_peak, hbm_src, w.name,
-                                     args.mode)
-            used = [host_gbs, hbm_gbs, alone_gbs]
-            if plan.host_fraction > 0:   # the side-by-side rates of this placement feed the next round
-                host_gbs, hbm_gbs = rates_of(meas)
-            rounds.append({"host_fraction": plan.host_fraction, "rates_used_gbs": used,
-                           "predicted_step_ms": plan.step_seconds * 1e3, "measured_step_ms": meas["ms"],
-                           "predicted_over_measured": plan.step_seconds * 1e3 / meas["ms"],
-                           "host_stream_gbs": rates_of(meas)[0] if plan.host_fraction > 0 else None,
-                           "hbm_split_k_gbs": rates_of(meas)[1]})
-            f_prev = plan.host_fraction
-        last = rounds[-1]
-        planner = {"rounds": rounds, "hbm_budget_bytes": budget if budget >= 0 else None,
-                   "hbm_alone_gbs": alone_gbs if alone_gbs > 0 else None, "all_hbm_step_ms": all_hbm_ms,
-                   "time_optimal_fraction": plan.time_optimal_fraction, "host_fraction": f_prev,
-                   "predicted_step_ms": last.get("predicted_step_ms"), "measured_step_ms": meas["ms"],
-                   "predicted_over_measured": last.get("predicted_over_measured"),
-                   "hbm_bytes_freed": float(kv.host_bytes), "hbm_bytes_used": float(kv.dev_bytes),
-                   "hbm_fraction_freed": kv.host_bytes / max(1, kv.host_bytes + kv.dev_bytes)}
+        planner, meas = plan_placement(dkv.dkv_plan_offload, measure_at, rates_of, x, budget, w.host_fraction, meas)
+        planner.update({"hbm_bytes_freed": float(kv.host_bytes), "hbm_bytes_used": float(kv.dev_bytes),
+                        "hbm_fraction_freed": kv.host_bytes / max(1, kv.host_bytes + kv.dev_bytes)})
     ms = meas["ms"]
     flush_buf = meas["flush_buf"]
 

@@ -91,3 +91,65 @@ def test_host_fraction_override_names_the_placement():
     assert bench.workload_for_rank("long_ctx", 1, 4096, 0.5).name == "long_ctx_ctx4096_h0.5"
     with pytest.raises(SystemExit):
         bench.parse_args(["--host-fraction", "1.5"])
+
+
+def _planner_model(alone_gbs, beside_far=2300.0, beside_near=4500.0, host_gbs=51.0):
+    """A modelled GPU: the host stream at host_gbs; the HBM kernel at alone_gbs with no host blocks, beside the
+    host stream slower, and slowest when the host stream dominates the step (f >= 0.5)."""
+    def measure(x, f):
+        hbm = alone_gbs if f == 0 else (beside_far if f >= 0.5 else beside_near)
+        t = x / (hbm * 1e9) if f == 0 else max(f * x / (host_gbs * 1e9), (1 - f) * x / (hbm * 1e9))
+        return {"ms": t * 1e3, "host": host_gbs if f > 0 else None, "hbm": hbm}
+    return measure
+
+
+def _plan(x, budget, f0, alone):
+    import decode_attention_host_b200 as dkv
+    model = _planner_model(alone)
+    seen = []
+
+    def measure_at(f):
+        seen.append(f)
+        return model(x, f)
+    rates = lambda m: (m["host"] if m["host"] is not None else 51.0 * 0.92, m["hbm"])  # noqa: E731
+    planner, meas = bench.plan_placement(dkv.dkv_plan_offload, measure_at, rates, x, budget, f0, model(x, f0))
+    return planner, meas, seen
+
+
+def test_planner_keeps_the_cache_in_hbm_when_the_kernel_alone_is_fastest():
+    x = 4.0 * (1 << 30)
+    planner, meas, seen = _plan(x, -1.0, 0.9, alone=5600.0)
+    # the whole cache in HBM, two side-by-side splits (from the far and then the near rates), then back
+    assert seen[0] == 0.0 and 0 < seen[1] < 0.05 and 0 < seen[2] < seen[1] and seen[-1] == 0.0
+    assert planner["host_fraction"] == 0.0 and planner["time_optimal_fraction"] == 0.0
+    assert planner["hbm_alone_gbs"] == 5600.0
+    assert abs(planner["predicted_over_measured"] - 1.0) < 1e-9
+    assert abs(meas["ms"] - x / 5600e9 * 1e3) < 1e-9
+
+
+def test_planner_splits_when_the_side_by_side_rate_wins():
+    x = 4.0 * (1 << 30)
+    planner, meas, seen = _plan(x, -1.0, 0.9, alone=3000.0)   # alone slower than 51 + 4500 side by side
+    f = planner["host_fraction"]
+    assert seen[0] == 0.0 and 0 < f < 0.05 and seen[-1] == f
+    assert abs(f - 51.0 / (51.0 + 4500.0)) < 1e-12           # settled on the near-point side-by-side rates
+    assert planner["rounds"][-1]["host_fraction"] == f
+    assert abs(planner["predicted_over_measured"] - 1.0) < 1e-9
+
+
+def test_planner_with_a_budget_never_measures_the_all_hbm_placement():
+    x = 4.0 * (1 << 30)
+    planner, meas, seen = _plan(x, 0.5 * x, 0.9, alone=5600.0)
+    assert seen == [0.5] and planner["hbm_alone_gbs"] is None
+    assert abs(planner["host_fraction"] - 0.5) < 1e-12
+    assert abs(planner["predicted_over_measured"] - 1.0) < 1e-9   # the model is exact at f >= 0.5
+
+
+def test_planner_on_a_workload_already_in_hbm():
+    """The workload's own placement is all-HBM: its measurement gives the alone rate; the side-by-side splits
+    are measured, lose to it, and the cache is rebuilt in HBM."""
+    x = 1.0 * (1 << 30)
+    planner, meas, seen = _plan(x, -1.0, 0.0, alone=5600.0)
+    assert planner["hbm_alone_gbs"] == 5600.0 and planner["host_fraction"] == 0.0
+    assert len(seen) == 3 and all(0 < f < 0.05 for f in seen[:2]) and seen[-1] == 0.0
+    assert abs(meas["ms"] - x / 5600e9 * 1e3) < 1e-9
