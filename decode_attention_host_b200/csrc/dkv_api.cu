@@ -102,7 +102,20 @@ constexpr bool kHostTma = DKV_HOST_TMA != 0;
 constexpr int kDevRefine = DKV_DEV_REFINE;
 constexpr int kDevUnitTokens = DKV_DEV_UNIT_TOKENS;
 static_assert(kDevRefine >= 1 && kDevRefine <= 8, "DKV_DEV_REFINE must be 1..8");
+// CTAs of the zero-copy host kernel when the configuration leaves it to the
+// library: every count from 4 to 24 keeps the PCIe link at 0.91-0.925 of the
+// copy engine's rate, but the HBM kernel beside it loses speed as the count
+// grows (its L2 shares the host kernel's long-latency sysmem reads: 4970,
+// 4800, 4490, 3780 GB/s with 4, 8, 16, 24 host CTAs).  A call whose host part
+// carries the step takes 16 (0.924 against 0.917 with 8 on a 90%-host step);
+// one whose host part is small against its HBM part takes 8 (a 99%-HBM
+// placement ran 0.93 ms against 1.39 ms).
 constexpr int kDefaultHostCtas = 16;
+constexpr int kLightHostCtas = 8;
+// The host part carries the step when its blocks are at least this share of
+// the HBM part's: B_pcie / B_hbm is about 1/100, so from 1/50 on the host
+// stream takes at least twice as long as the HBM kernel.
+constexpr int kHostCarriesDenominator = 50;
 constexpr int kListThreads = 1024;  // threads of the pool-lists kernel
 
 // cudaMalloc, or a simulated out-of-memory failure when the test hook
@@ -206,7 +219,7 @@ struct dkv_handle {
   int units_target = 0;       // warps of the widest split launch (one resident wave: 2 CTAs per SM)
   size_t part_rows = 0;
   float qscale = 0.f;
-  int host_ctas = 0;
+  int host_ctas = 0;           // the configuration's count; 0: chosen per call
   float* part_o = nullptr;
   float* part_lse = nullptr;
   int32_t* status = nullptr;
@@ -275,17 +288,24 @@ void release(dkv_handle* h) {
 }
 
 // Warps a split launch can keep resident: 2 CTAs of kWarps warps per SM, less
-// the SMs' share the zero-copy host kernel holds while it runs beside it.
-long launch_warps(const dkv_handle* h, bool beside_host) {
-  const long ctas = 2L * h->sm_count - (beside_host ? static_cast<long>(h->host_ctas) * (2 - h->beside_host) : 0);
+// the SMs' share the zero-copy host kernel's host_ctas CTAs hold while it runs
+// beside it (host_ctas = 0: it does not).
+long launch_warps(const dkv_handle* h, int host_ctas) {
+  const long ctas = 2L * h->sm_count - static_cast<long>(host_ctas) * (2 - h->beside_host);
   return dkv::kWarps * (ctas > 1 ? ctas : 1);
+}
+
+// CTAs of the zero-copy host kernel for a call with these pool sizes.
+int call_host_ctas(const dkv_handle* h, long long host_blocks, long long dev_blocks) {
+  if (h->host_ctas > 0) return h->host_ctas;
+  return host_blocks * kHostCarriesDenominator >= dev_blocks ? kDefaultHostCtas : kLightHostCtas;
 }
 
 // Split plan of the HBM kernel of a call whose blocks all sit in HBM (the
 // only split launch of the call).
 dkv::SplitPlan alone_plan(const dkv_handle* h, int nblk, int batch) {
   const long per = static_cast<long>(batch) * h->cfg.num_kv_heads;
-  return dkv::plan_split_refined(nblk, per, h->cfg.block_size, launch_warps(h, false),
+  return dkv::plan_split_refined(nblk, per, h->cfg.block_size, launch_warps(h, 0),
                                  batch < 2 ? 1 : kDevRefine, kDevUnitTokens);
 }
 
@@ -391,7 +411,7 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   const bool bf16 = c.kv_dtype == DKV_KV_BF16;
   const double scale = c.scale > 0.0 ? c.scale : 1.0 / std::sqrt(static_cast<double>(c.head_dim));
   h->qscale = static_cast<float>(scale * 1.4426950408889634);  // * log2(e)
-  h->host_ctas = c.host_ctas > 0 ? c.host_ctas : kDefaultHostCtas;
+  h->host_ctas = c.host_ctas;
   const bool rope = c.rope_base > 0.0;
   h->host_kernel = pick_split<kHostStages, kHostTma>(c.head_dim, G, bf16, rope);
   h->dev_kernel = pick_split<kDevStages, false>(c.head_dim, G, bf16, rope);
@@ -408,7 +428,7 @@ int dkv_create(const dkv_config* cfg, dkv_handle** out) {
   h->beside_host = fits_beside(h->host_kernel.ptr, split_smem(c.head_dim, kHostStages),
                                (kDevTmaMode == 0 ? h->dev_kernel : h->dev_tma_kernel).ptr,
                                split_smem(c.head_dim, kDevStages), c.device);
-  h->units_target = static_cast<int>(launch_warps(h, false));
+  h->units_target = static_cast<int>(launch_warps(h, 0));
   // partial rows: batch * Tq * Hq * (host splits + device splits), each launch's
   // splits <= max(1, units_target / (batch * Hkv)); Tq * G <= 16 rows per unit
   // (multi-token queries) and batch * Tq <= max_batch
@@ -560,9 +580,10 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
   const bool use_lists = run_host && run_dev;    // each launch walks the list of its own pool's blocks
   const int nblk_cap = block_table_stride < c.max_blocks_per_seq ? block_table_stride : c.max_blocks_per_seq;
   const long per = static_cast<long>(batch) * c.num_kv_heads;
-  const long host_warps = staged ? launch_warps(h, false) : static_cast<long>(dkv::kWarps) * h->host_ctas;
+  const int host_ctas = concurrent ? call_host_ctas(h, host_split, num_dev_blocks) : 0;
+  const long host_warps = staged ? launch_warps(h, 0) : static_cast<long>(dkv::kWarps) * host_ctas;
   const dkv::SplitPlan ph = dkv::plan_split(nblk_cap, per, c.block_size, host_warps, 0);
-  const dkv::SplitPlan pd = run_host ? dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, concurrent), 0)
+  const dkv::SplitPlan pd = run_host ? dkv::plan_split(nblk_cap, per, c.block_size, launch_warps(h, host_ctas), 0)
                                       : alone_plan(h, nblk_cap, batch);
   const int nsplit_h = run_host ? ph.nsplit : 0;
   const int nsplit_d = run_dev ? pd.nsplit : 0;
@@ -667,7 +688,7 @@ int decode_impl(dkv_handle* h, const float* q, const void* k_host, const void* v
     if (kHostTma && !multi && (rc = pool_maps(h, h->host_maps, k_host, v_host, host_split, &hmaps)) != DKV_OK)
       return rc;
     if ((rc = prof_mark(h, 0, h->aux, false)) != DKV_OK) return rc;
-    host_k.fn(dim3(ctas_for(hp, h->host_ctas)), host_smem, h->aux, hp, *hmaps);
+    host_k.fn(dim3(ctas_for(hp, host_ctas)), host_smem, h->aux, hp, *hmaps);
     DKV_CUDA(cudaGetLastError());
     if ((rc = prof_mark(h, 0, h->aux, true)) != DKV_OK) return rc;
     DKV_CUDA(cudaEventRecord(h->ev_join, h->aux));

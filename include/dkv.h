@@ -70,7 +70,10 @@ typedef struct dkv_config {
   int32_t max_batch;          /* largest batch passed to dkv_attn_decode */
   int32_t max_blocks_per_seq; /* largest number of blocks of one sequence */
   int32_t device;             /* CUDA device ordinal the handle is bound to */
-  int32_t host_ctas;          /* CTAs of the zero-copy host kernel; 0 = library default (16) */
+  int32_t host_ctas;          /* CTAs of the zero-copy host kernel; 0 = chosen per call:
+                                 16 while the host pool holds at least 1/50 of the device
+                                 pool's blocks (the host stream carries the step), else 8
+                                 (the HBM kernel beside it keeps more of its speed) */
 } dkv_config;
 
 typedef struct dkv_handle dkv_handle;

@@ -226,6 +226,22 @@ def test_full_size_all_in_hbm_sampled_against_oracle(name, groups):
     case.free()
 
 
+@pytest.mark.parametrize("host_fraction", [0.01, 0.03])
+def test_small_host_share_full_size_sampled(host_fraction):
+    """A placement near the offload planner's balance point: 1% (light host stream of 8 CTAs beside an HBM
+    launch planned for the warps it leaves) and 3% (16 CTAs) of the 64k cell's blocks on the host."""
+    w = kvgen.get("sweep_L65536_f0").replace(name=f"sweep_L65536_f{host_fraction:g}", host_fraction=host_fraction)
+    case = gc.Case(w)
+    got = case.run()
+    assert np.isfinite(got).all()
+    assert case.attn.status() == 0 and case.kv.host_split > 0 and case.attn.launches() == 4
+    mask = gc.sampled_groups(w, 3, 77)
+    err = gc.sampled_err(w, got, case.oracle(group_mask=mask), mask)
+    gc.record("test_small_host_share_full_size_sampled", w.name, err, f"{int(mask.sum())} of {mask.size}")
+    assert err <= gc.TOL, f"{w.name}: {err:.3e}"
+    case.free()
+
+
 @pytest.mark.parametrize("cell", [c.name for c in kvgen.sweep_cells()])
 def test_every_sweep_cell_full_size_sampled(cell):
     """All 20 context x host-fraction cells at full size (B=4, 1% outlier keys x8), in the bench's launch
