@@ -85,14 +85,13 @@ constexpr int kDevTmaMode = DKV_DEV_TMA;
 constexpr bool kHostTma = DKV_HOST_TMA != 0;
 // Units per resident warp of the HBM kernel (single- or multi-token) when all
 // blocks sit in HBM and the batch holds 2 or more sequences (build-time
-// knobs): up to
-// DKV_DEV_REFINE (1 to 8; the partial-row workspace covers 8) while each unit
-// keeps at least DKV_DEV_UNIT_TOKENS tokens.  With ragged lengths the plan,
-// sized by the table capacity, otherwise gives the longest sequences units as
-// long as a warp's whole share (an all-HBM batch of 16 sequences of 1k-16k
-// tokens ran 1.9x faster with 2 units per warp, with 4 query tokens 1.95x);
-// uniform batches are unchanged within 1%.  One sequence cannot be ragged and keeps one unit per
-// warp.
+// knobs): up to DKV_DEV_REFINE (1 to 8; the partial-row workspace covers 8)
+// while each unit keeps at least DKV_DEV_UNIT_TOKENS tokens.  With ragged
+// lengths the plan, sized by the table capacity, otherwise gives the longest
+// sequences units as long as a warp's whole share (an all-HBM batch of 16
+// sequences of 1k-16k tokens ran 1.9x faster with 2 units per warp, with 4
+// query tokens 1.95x); uniform batches are unchanged within 1%.  One sequence
+// cannot be ragged and keeps one unit per warp.
 #ifndef DKV_DEV_REFINE
 #define DKV_DEV_REFINE 2
 #endif
@@ -108,8 +107,8 @@ static_assert(kDevRefine >= 1 && kDevRefine <= 8, "DKV_DEV_REFINE must be 1..8")
 // grows (its L2 shares the host kernel's long-latency sysmem reads: 4970,
 // 4800, 4490, 3780 GB/s with 4, 8, 16, 24 host CTAs).  A call whose host part
 // carries the step takes 16 (0.924 against 0.917 with 8 on a 90%-host step);
-// one whose host part is small against its HBM part takes 8 (a 99%-HBM
-// placement ran 0.93 ms against 1.39 ms).
+// one whose host part is small against its HBM part takes 8 (long_ctx
+// planned for a 99% HBM budget ran 1.00 ms against 1.31 ms).
 constexpr int kDefaultHostCtas = 16;
 constexpr int kLightHostCtas = 8;
 // The host part carries the step when its blocks are at least this share of
