@@ -107,9 +107,10 @@ static_assert(kDevRefine >= 1 && kDevRefine <= 8, "DKV_DEV_REFINE must be 1..8")
 // grows (its L2 shares the host kernel's long-latency sysmem reads: 4970,
 // 4800, 4490, 3780 GB/s with 4, 8, 16, 24 host CTAs).  A call whose host part
 // carries the step takes 16 (0.924 against 0.917 with 8 on a 90%-host step);
-// one whose host part is small against its HBM part takes 8 (a 1M-token
-// sequence, 4 GiB of KV, with 1% of its blocks on the host: 1.00 ms against
-// 1.31 ms).
+// one whose host part is small against its HBM part takes 8 (for a 1M-token
+// sequence, 4 GiB of KV, the planned placement under a 99% HBM budget then
+// ran 1.00 ms, with 1.1% of the blocks on the host, against 1.31 ms with 16
+// host CTAs, with 1.5%).
 constexpr int kDefaultHostCtas = 16;
 constexpr int kLightHostCtas = 8;
 // The host part carries the step when its blocks are at least this share of
