@@ -217,8 +217,10 @@ DKV_API int dkv_last_launch_count(const dkv_handle* h, int32_t* count);
  * kernel; with 2 or more sequences, at 2 units per warp when every unit still
  * holds at least 1024 tokens (finer units keep ragged batches balanced).
  * With host blocks as well, each launch splits the list of its own pool's
- * blocks of every sequence, and the HBM launch plans one unit per warp left
- * beside the zero-copy host kernel. */
+ * blocks of every sequence, and the HBM launch plans for the warps left beside
+ * the zero-copy host kernel: one unit per warp while the host part carries the
+ * step, two (under the same conditions as above) when the host pool holds
+ * less than 1/50 of the device pool's blocks. */
 DKV_API int dkv_query_plan(const dkv_handle* h, int32_t batch, int32_t block_table_stride, int32_t* num_splits,
                    int32_t* blocks_per_split);
 
