@@ -55,9 +55,10 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long_ctx")
     ap.add_argument("--impl", choices=("dkv", "reference"), default="dkv")
-    ap.add_argument("--mode", choices=("zero_copy", "staged", "planned"), default="zero_copy",
+    ap.add_argument("--mode", choices=("zero_copy", "staged", "planned", "append"), default="zero_copy",
                     help="staged: the prefetch comparator (host pool copied into HBM each step); "
-                         "planned: the placement chosen by the offload planner from measured rates")
+                         "planned: the placement chosen by the offload planner from measured rates; "
+                         "append: the write side, K/V projection of every sequence's new token and its store")
     ap.add_argument("--hbm-budget-frac", type=float, default=-1.0,
                     help="planned mode: HBM the cache may use, as a fraction of its bytes (< 0: unlimited)")
     ap.add_argument("--queries", type=int, default=1,
@@ -625,11 +626,100 @@ def run_dkv(args):
     return 0
 
 
+def append_bytes(w: kvgen.Workload, hidden: int, dev_stores: int, host_stores: int) -> tuple[int, int]:
+    """Algorithmic bytes of one append step: (HBM bytes, host bytes).  HBM: the two weight matrices
+    [Hkv*D][hidden] (16-bit), the fp32 hidden states and the K/V rows stored into device blocks; host: the K/V
+    rows stored into host blocks (over PCIe)."""
+    rows = w.num_kv_heads * w.head_dim
+    row_bytes = 2 * rows * 2                      # one token's K and V, 16-bit
+    return 2 * rows * hidden * 2 + w.batch * hidden * 4 + dev_stores * row_bytes, host_stores * row_bytes
+
+
+def run_append(args):
+    """--mode append: the K/V projection of each sequence's new token (hidden = Hq * D, the model width of the
+    named workloads) and its store into the block holding position L - 1 of the workload's own cache, timed
+    like a decode step.  HBM-bound: the weights are read once per step."""
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init("nccl")
+    import decode_attention_host_b200 as dkv
+
+    w = workload_for_rank(args.workload, rank, args.ctx, args.host_fraction)
+    lens = kvgen.gen_seq_lens(w)
+    lmax = max(1, int(lens.max(initial=0)))
+    zeros = np.zeros((w.batch, w.num_kv_heads, lmax, w.head_dim), dtype=np.uint16)   # contents do not matter here
+    placement = dkv.DKV_PLACE_PREFIX_HOST if w.placement == "prefix_host" else dkv.DKV_PLACE_RANDOM
+    kv = dkv.PagedKV(zeros, zeros, lens, w.block_size, placement, w.host_fraction, w.shuffle, w.seed, device=local)
+    del zeros
+    attn = dkv.DecodeAttention(w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                               dkv.DKV_KV_BF16 if w.kv_dtype == kvgen.BF16 else dkv.DKV_KV_F16, w.rope_base,
+                               w.batch, kv.stride, device=local, host_ctas=args.host_ctas)
+    hidden = w.num_q_heads * w.head_dim
+    wdt = torch.bfloat16 if w.kv_dtype == kvgen.BF16 else torch.float16
+    gen = torch.Generator(device=device).manual_seed(w.seed)
+    x = torch.randn(w.batch, hidden, device=device, generator=gen)
+    w_k = (torch.randn(w.num_kv_heads * w.head_dim, hidden, device=device, generator=gen) * hidden ** -0.5).to(wdt)
+    w_v = (torch.randn(w.num_kv_heads * w.head_dim, hidden, device=device, generator=gen) * hidden ** -0.5).to(wdt)
+    # the new token overwrites position L - 1, which the table covers (the timed quantity does not depend on it)
+    pos = np.maximum(lens - 1, 0)
+    kv.seq_lens_dev.copy_(torch.from_numpy(pos.astype(np.int32)))
+    ids = kv.table[np.arange(w.batch), pos // w.block_size]
+    live = lens > 0
+    host_stores = int(np.count_nonzero(live & (ids < kv.host_split)))
+    dev_stores = int(np.count_nonzero(live)) - host_stores
+    hbm_bytes, host_bytes = append_bytes(w, hidden, dev_stores, host_stores)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        attn.append(x, w_k, w_v, kv, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if attn.status() != 0:
+        raise RuntimeError("device status nonzero after warm-up")
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)   # the weights fit in L2
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier()
+    torch.cuda.synchronize(device)
+    clocks.start()
+    ms_local = timed_steps(step, args.steps, stream, flush_buf)
+    torch.cuda.synchronize(device)
+    clock_info = clocks.stop()
+    barrier()
+    ms = max_over_ranks(ms_local, device)
+    peaks = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    hbm_src = "MEASURED_PEAKS.json hbm_gbs (copy, measured)" if "hbm_gbs" in peaks else "fallback 6650 GB/s"
+    achieved = hbm_bytes / (ms * 1e-3) / 1e9
+    total = (hbm_bytes + host_bytes) * world
+    if rank == 0:
+        line = {
+            "metric": "KV append: K/V projection of the new token and its store, µs/step & GB/s", "value":
+            total / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+            "config": dict(workload_config(w, world), mode="append", hidden=hidden, hbm_bytes=hbm_bytes,
+                           host_bytes=host_bytes, host_stores=host_stores, dev_stores=dev_stores,
+                           l2="L2 flushed between timed steps (%d MiB write outside the step events): "
+                              "%.1f MiB of weights per step" % (FLUSH_BYTES >> 20, hbm_bytes / 2**20)),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "peak_source": hbm_src, "traffic": None},
+            "e2e": None, "gpu_launches": args.steps, "clocks": clock_info, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    kv.free()
+    attn.close()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
-    rc = run_dkv(args)
+    rc = run_append(args) if args.mode == "append" else run_dkv(args)
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
         dist.destroy_process_group()

@@ -191,6 +191,34 @@ SplitEntry pick_multi(int D, bool bf16, bool rope) {
 // shared memory of the multi-token kernel: per warp a 2-stage (K, V) ring and one rotated-K lo tile
 size_t multi_smem(int D) { return dkv::multi_smem_bytes(D); }
 
+// The append kernel for `nb` sequences per pass (1, 2, 4, 8 or 16).
+template <bool BF16, int NB>
+cudaError_t launch_append_nb(dim3 grid, cudaStream_t s, const dkv::AppendParams& ap) {
+  const size_t smem = dkv::append_smem_bytes(NB);
+  if (smem > 48 * 1024) {
+    // once per process and instance (the attribute holds for every device)
+    static const cudaError_t set = cudaFuncSetAttribute(dkv::append_kernel<BF16, NB>,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        static_cast<int>(smem));
+    if (set != cudaSuccess) return set;
+  }
+  dkv::append_kernel<BF16, NB><<<grid, dkv::kAppendWarps * 32, smem, s>>>(ap);
+  return cudaGetLastError();
+}
+template <bool BF16>
+cudaError_t launch_append_t(int nb, dim3 grid, cudaStream_t s, const dkv::AppendParams& ap) {
+  switch (nb) {
+    case 1: return launch_append_nb<BF16, 1>(grid, s, ap);
+    case 2: return launch_append_nb<BF16, 2>(grid, s, ap);
+    case 4: return launch_append_nb<BF16, 4>(grid, s, ap);
+    case 8: return launch_append_nb<BF16, 8>(grid, s, ap);
+    default: return launch_append_nb<BF16, dkv::kAppendBatch>(grid, s, ap);
+  }
+}
+cudaError_t launch_append(bool bf16, int nb, dim3 grid, cudaStream_t s, const dkv::AppendParams& ap) {
+  return bf16 ? launch_append_t<true>(nb, grid, s, ap) : launch_append_t<false>(nb, grid, s, ap);
+}
+
 // The merge, optionally as a programmatic dependent launch of the split kernel
 // just before it on the stream: its grid is set up while that kernel drains
 // and its first instruction waits for that kernel's results.
@@ -813,11 +841,9 @@ int dkv_append_kv(dkv_handle* h, const float* x, const void* w_k, const void* w_
   ap.max_len = (block_table_stride < c.max_blocks_per_seq ? block_table_stride : c.max_blocks_per_seq) * c.block_size;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(2 * c.num_kv_heads * c.head_dim / dkv::kAppendRows);
-  if (c.kv_dtype == DKV_KV_BF16)
-    dkv::append_kernel<true><<<grid, dkv::kAppendRows * 32, 0, s>>>(ap);
-  else
-    dkv::append_kernel<false><<<grid, dkv::kAppendRows * 32, 0, s>>>(ap);
-  DKV_CUDA(cudaGetLastError());
+  // sequences per pass: the smallest of 1, 2, 4, 8, 16 that covers the batch (16 for larger batches)
+  const int nb = batch > 8 ? dkv::kAppendBatch : batch > 4 ? 8 : batch > 2 ? 4 : batch;
+  DKV_CUDA(launch_append(c.kv_dtype == DKV_KV_BF16, nb, grid, s, ap));
   return DKV_OK;
 }
 

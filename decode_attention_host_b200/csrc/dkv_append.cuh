@@ -9,10 +9,13 @@
 // holds position seq_lens[b], in the host or the device pool.
 //
 // The product is bound by the weight bytes (batch is small), so it runs on the
-// CUDA cores: one warp per output row reads the weight row once with 16-byte
-// loads and applies it to every sequence; a CTA covers 8 consecutive rows
-// (8 dims of one head), so each sequence's 8 results leave as one 16-byte
-// store -- over PCIe when the block is host-resident.
+// CUDA cores.  A CTA owns 8 consecutive output rows (8 dims of one head), so
+// each sequence's 8 results leave as one 16-byte store -- over PCIe when the
+// block is host-resident.  Its 8 warps split the hidden dimension: in each
+// warp, 4 lanes share a row and read a 64-byte run of it (16 bytes each), the
+// 8 rows side by side; every weight byte is read once for up to 16
+// sequences, whose hidden states the CTA stages in shared memory.  Lane
+// partials are combined by shuffles, the warps' through shared memory.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -22,8 +25,9 @@
 
 namespace dkv {
 
-constexpr int kAppendRows = 8;                 // output rows per CTA (one warp each)
-constexpr int kAppendBatch = 8;                // sequences per pass over a weight row
+constexpr int kAppendRows = 8;                 // output rows per CTA
+constexpr int kAppendWarps = 8;                // warps per CTA, each over part of the hidden dimension
+constexpr int kAppendBatch = 16;               // sequences per pass over the weights
 
 struct AppendParams {
   const float* x;           // [B][H]
@@ -66,59 +70,59 @@ __device__ __forceinline__ void widen8(const uint4& u, float (&w)[8]) {
   }
 }
 
-// grid.x = 2*Hkv*D / 8 ; block = 8 warps
-template <bool BF16>
-__global__ void __launch_bounds__(kAppendRows * 32) append_kernel(const AppendParams p) {
-  __shared__ __align__(16) uint16_t s_out[kAppendBatch][kAppendRows];
+// Columns a CTA's lanes cover in one step (8 warps x 4 lanes x 8 columns).
+constexpr int kAppendStep = kAppendWarps * 4 * 8;
+
+// Steps per stage of x in shared memory for NB sequences per pass: the more
+// sequences, the more work per weight byte hides the loads' latency, so the
+// fewer weight loads need to be in flight per lane (one stage's worth).
+__host__ __device__ constexpr int append_group(int nb) { return nb <= 2 ? 16 : (nb <= 4 ? 8 : 4); }
+
+// Dynamic shared memory of append_kernel<*, NB>: x of NB sequences over one
+// stage of columns.
+__host__ __device__ constexpr size_t append_smem_bytes(int nb) {
+  return static_cast<size_t>(nb) * kAppendStep * append_group(nb) * sizeof(float);
+}
+
+// grid.x = 2*Hkv*D / kAppendRows; block = kAppendWarps warps.  NB: sequences
+// per pass over the weights (1, 2, 4, 8 or 16, the smallest that covers the
+// batch up to 16), so that a small batch issues no work for absent sequences.
+// The hidden dimension is walked in stages of kGroup steps: each lane first
+// issues its weight loads of the stage, then the CTA stages x of those
+// columns in shared memory (every lane of a row reads it there, not from L2),
+// so the two latencies overlap.
+template <bool BF16, int NB>
+__global__ void __launch_bounds__(kAppendWarps * 32, 2) append_kernel(const AppendParams p) {
+  static_assert(NB >= 1 && NB <= kAppendBatch, "1..16 sequences per pass");
+  constexpr int kGroup = append_group(NB);          // steps per stage
+  constexpr int kAppendCols = kAppendStep * kGroup; // columns per stage
+  extern __shared__ __align__(16) float s_x[];  // [NB][kAppendCols]
+  __shared__ float s_part[kAppendWarps][NB][kAppendRows];
+  __shared__ __align__(16) uint16_t s_out[NB][kAppendRows];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int r = lane >> 2;                          // row of this lane among the CTA's 8
+  const int q = lane & 3;                           // its 16-byte column in the row's 64-byte run
   const int rows_kv = p.hkv * p.head_dim;
   const int row0 = blockIdx.x * kAppendRows;        // first output row of this CTA
   const bool is_v = row0 >= rows_kv;
   const int r_local = row0 - (is_v ? rows_kv : 0);  // row inside W_k or W_v
   const int h = r_local / p.head_dim;
   const int d0 = r_local % p.head_dim;              // multiple of 8
-  const uint16_t* wrow = (is_v ? p.w_v : p.w_k) + static_cast<size_t>(r_local + warp) * p.hidden;
+  const uint16_t* wrow = (is_v ? p.w_v : p.w_k) + static_cast<size_t>(r_local + r) * p.hidden;
+  const int col = (warp * 4 + q) * 8;               // this lane's 8 columns inside a step
+  auto load_w = [&](int c) {
+    return c < p.hidden ? *reinterpret_cast<const uint4*>(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+  };
 
-  for (int b0 = 0; b0 < p.batch; b0 += kAppendBatch) {
-    const int nb = min(kAppendBatch, p.batch - b0);
-    float acc[kAppendBatch];
-#pragma unroll
-    for (int i = 0; i < kAppendBatch; ++i) acc[i] = 0.f;
-    for (int c = lane * 8; c < p.hidden; c += 32 * 8) {
-      float w[8];
-      widen8<BF16>(*reinterpret_cast<const uint4*>(wrow + c), w);
-#pragma unroll
-      for (int i = 0; i < kAppendBatch; ++i) {
-        if (i < nb) {
-          const float* xr = p.x + static_cast<size_t>(b0 + i) * p.hidden + c;
-          const float4 x0 = __ldg(reinterpret_cast<const float4*>(xr));
-          const float4 x1 = __ldg(reinterpret_cast<const float4*>(xr + 4));
-          float a = acc[i];
-          a = fmaf(w[0], x0.x, a);
-          a = fmaf(w[1], x0.y, a);
-          a = fmaf(w[2], x0.z, a);
-          a = fmaf(w[3], x0.w, a);
-          a = fmaf(w[4], x1.x, a);
-          a = fmaf(w[5], x1.y, a);
-          a = fmaf(w[6], x1.z, a);
-          a = fmaf(w[7], x1.w, a);
-          acc[i] = a;
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kAppendBatch; ++i) {
-      float a = acc[i];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0 && i < nb) s_out[i][warp] = round16<BF16>(a);
-    }
-    __syncthreads();
+  for (int b0 = 0; b0 < p.batch; b0 += NB) {
+    const int nb = min(NB, p.batch - b0);
+    // destination of sequence b0 + threadIdx.x (threads < nb), looked up while
+    // the projection runs: its position, the table entry, the pool
+    uint16_t* dst = nullptr;
     if (threadIdx.x < nb) {
       const int b = b0 + threadIdx.x;
       const int L = p.seq_lens[b];  // position of the new token
-      uint16_t* dst = nullptr;
       if (L < 0 || L >= p.max_len) {
         atomicOr(p.status, 2);
       } else {
@@ -134,11 +138,69 @@ __global__ void __launch_bounds__(kAppendRows * 32) append_kernel(const AppendPa
         } else {
           atomicOr(p.status, 1);
         }
-        if (pool)
-          dst = pool + ((blk * p.hkv + h) * p.block_size + (L % p.block_size)) * p.head_dim + d0;
+        if (pool) dst = pool + ((blk * p.hkv + h) * p.block_size + (L % p.block_size)) * p.head_dim + d0;
       }
-      if (dst) *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&s_out[threadIdx.x][0]);
     }
+    // per sequence, even and odd columns accumulate in the two halves of a
+    // packed pair (one f32x2 FMA per two columns)
+    float2 acc[NB];
+#pragma unroll
+    for (int i = 0; i < NB; ++i) acc[i] = make_float2(0.f, 0.f);
+    for (int g0 = 0; g0 < p.hidden; g0 += kAppendCols) {
+      // this lane's weights of the stage, in flight while x is staged
+      uint4 raw[kGroup];
+#pragma unroll
+      for (int u = 0; u < kGroup; ++u) raw[u] = load_w(g0 + col + u * kAppendStep);
+      // x of this stage (zeros for absent sequences and past the hidden size)
+      for (int e = threadIdx.x * 4; e < NB * kAppendCols; e += kAppendWarps * 32 * 4) {
+        const int i = e / kAppendCols, cc = e % kAppendCols;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < nb && g0 + cc < p.hidden)
+          v = __ldg(reinterpret_cast<const float4*>(p.x + static_cast<size_t>(b0 + i) * p.hidden + g0 + cc));
+        *reinterpret_cast<float4*>(s_x + e) = v;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < kGroup; ++u) {
+        float w[8];
+        widen8<BF16>(raw[u], w);   // zeros past the hidden size
+        const float2 w01 = make_float2(w[0], w[1]), w23 = make_float2(w[2], w[3]);
+        const float2 w45 = make_float2(w[4], w[5]), w67 = make_float2(w[6], w[7]);
+        const int cs = col + u * kAppendStep;   // column inside the stage
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          const float4 x0 = *reinterpret_cast<const float4*>(s_x + i * kAppendCols + cs);
+          const float4 x1 = *reinterpret_cast<const float4*>(s_x + i * kAppendCols + cs + 4);
+          float2 a = acc[i];
+          a = __ffma2_rn(w01, make_float2(x0.x, x0.y), a);
+          a = __ffma2_rn(w23, make_float2(x0.z, x0.w), a);
+          a = __ffma2_rn(w45, make_float2(x1.x, x1.y), a);
+          a = __ffma2_rn(w67, make_float2(x1.z, x1.w), a);
+          acc[i] = a;
+        }
+      }
+      __syncthreads();   // before the next stage overwrites s_x
+    }
+    // the 4 lanes of a row, then the warps
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+      float a = acc[i].x + acc[i].y;
+      a += __shfl_xor_sync(0xffffffffu, a, 1);
+      a += __shfl_xor_sync(0xffffffffu, a, 2);
+      if (q == 0) s_part[warp][i][r] = a;
+    }
+    __syncthreads();
+    if (threadIdx.x < NB * kAppendRows) {
+      const int i = threadIdx.x / kAppendRows, rr = threadIdx.x % kAppendRows;
+      if (i < nb) {
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < kAppendWarps; ++w) a += s_part[w][i][rr];
+        s_out[i][rr] = round16<BF16>(a);
+      }
+    }
+    __syncthreads();
+    if (dst) *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&s_out[threadIdx.x][0]);
     __syncthreads();
   }
 }

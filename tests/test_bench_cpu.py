@@ -153,3 +153,12 @@ def test_planner_on_a_workload_already_in_hbm():
     assert planner["hbm_alone_gbs"] == 5600.0 and planner["host_fraction"] == 0.0
     assert len(seen) == 3 and all(0 < f < 0.05 for f in seen[:2]) and seen[-1] == 0.0
     assert abs(meas["ms"] - x / 5600e9 * 1e3) < 1e-9
+
+
+def test_append_bytes_count_weights_states_and_stores():
+    import kvgen
+    w = kvgen.get("llama3_8b")             # Hkv*D = 1024 rows, 8 sequences
+    hbm, host = bench.append_bytes(w, 4096, dev_stores=5, host_stores=3)
+    assert hbm == 2 * 1024 * 4096 * 2 + 8 * 4096 * 4 + 5 * 2 * 1024 * 2
+    assert host == 3 * 2 * 1024 * 2
+    assert bench.parse_args(["--mode", "append"]).mode == "append"

@@ -17,6 +17,10 @@ from tests import gpu_cases as gc
 pytestmark = pytest.mark.gpu
 
 
+def w_batch(kw) -> int:
+    return kw["batch"]
+
+
 def _exact_round(y: np.ndarray, kv_dtype: str) -> np.ndarray:
     """fp64 -> value of the nearest 16-bit number (ties to even), computed exactly."""
     bits = 8 if kv_dtype == kvgen.BF16 else 11
@@ -76,9 +80,13 @@ def _stored(case, w, b, pos, which):
 @pytest.mark.parametrize("name,kw,hidden", [
     ("llama3_8b", dict(batch=5, ctx=(40, 700), block_size=16), 512),
     ("opt_6_7b", dict(batch=3, ctx=(1, 300)), 256),
+    # 16 sequences per pass over the weights: one full pass, then a pass of 4 more; a hidden size that is
+    # not a multiple of the 256 columns a CTA covers per step
+    ("llama3_8b", dict(batch=20, ctx=(10, 200), block_size=16), 4104),
+    ("tiny_gqa", dict(batch=12, ctx=(1, 100)), 264),
 ])
 def test_projection_is_stored_rounded_at_its_position(name, kw, hidden):
-    w = kvgen.get(name).replace(name=f"append_{name}", **kw)
+    w = kvgen.get(name).replace(name=f"append_{name}_{w_batch(kw)}", **kw)
     case, lens, x, wk, wv = _setup(w, hidden, 50)
     before_k = [_stored(case, w, b, int(lens[b]) - 1, "k") for b in range(w.batch) if lens[b] > 0]
     _append(case, lens, x, wk, wv)
