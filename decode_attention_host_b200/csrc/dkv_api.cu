@@ -840,9 +840,9 @@ int dkv_append_kv(dkv_handle* h, const float* x, const void* w_k, const void* w_
   ap.num_dev_blocks = num_dev_blocks;
   ap.max_len = (block_table_stride < c.max_blocks_per_seq ? block_table_stride : c.max_blocks_per_seq) * c.block_size;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const dim3 grid(2 * c.num_kv_heads * c.head_dim / dkv::kAppendRows);
   // sequences per pass: the smallest of 1, 2, 4, 8, 16 that covers the batch (16 for larger batches)
   const int nb = batch > 8 ? dkv::kAppendBatch : batch > 4 ? 8 : batch > 2 ? 4 : batch;
+  const dim3 grid(2 * c.num_kv_heads * c.head_dim / dkv::append_cta_rows(nb));
   DKV_CUDA(launch_append(c.kv_dtype == DKV_KV_BF16, nb, grid, s, ap));
   return DKV_OK;
 }

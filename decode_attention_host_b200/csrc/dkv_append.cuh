@@ -25,7 +25,7 @@
 
 namespace dkv {
 
-constexpr int kAppendRows = 8;                 // output rows per CTA
+constexpr int kAppendRows = 8;                 // rows one lane of each of 8 row slots covers per CTA
 constexpr int kAppendWarps = 8;                // warps per CTA, each over part of the hidden dimension
 constexpr int kAppendBatch = 16;               // sequences per pass over the weights
 
@@ -78,47 +78,57 @@ constexpr int kAppendStep = kAppendWarps * 4 * 8;
 // fewer weight loads need to be in flight per lane (one stage's worth).
 __host__ __device__ constexpr int append_group(int nb) { return nb <= 2 ? 16 : (nb <= 4 ? 8 : 4); }
 
+// Rows per lane: with 16 sequences per pass a lane takes two rows (16 per
+// CTA), so x is staged once for twice the weight bytes.
+__host__ __device__ constexpr int append_rows_per_lane(int nb) { return nb >= 16 ? 2 : 1; }
+
+// Output rows per CTA (8 or 16 dims of one head; head_dim is 64 or 128).
+__host__ __device__ constexpr int append_cta_rows(int nb) { return kAppendRows * append_rows_per_lane(nb); }
+
 // Dynamic shared memory of append_kernel<*, NB>: x of NB sequences over one
 // stage of columns.
 __host__ __device__ constexpr size_t append_smem_bytes(int nb) {
   return static_cast<size_t>(nb) * kAppendStep * append_group(nb) * sizeof(float);
 }
 
-// grid.x = 2*Hkv*D / kAppendRows; block = kAppendWarps warps.  NB: sequences
-// per pass over the weights (1, 2, 4, 8 or 16, the smallest that covers the
-// batch up to 16), so that a small batch issues no work for absent sequences.
-// The hidden dimension is walked in stages of kGroup steps: each lane first
-// issues its weight loads of the stage, then the CTA stages x of those
-// columns in shared memory (every lane of a row reads it there, not from L2),
-// so the two latencies overlap.
+// grid.x = 2*Hkv*D / append_cta_rows(NB); block = kAppendWarps warps.  NB:
+// sequences per pass over the weights (1, 2, 4, 8 or 16, the smallest that
+// covers the batch up to 16), so that a small batch issues no work for absent
+// sequences.  The hidden dimension is walked in stages of kGroup steps: each
+// lane first issues its weight loads of the stage, then the CTA stages x of
+// those columns in shared memory (every lane of a row reads it there, not
+// from L2), so the two latencies overlap.
 template <bool BF16, int NB>
 __global__ void __launch_bounds__(kAppendWarps * 32, 2) append_kernel(const AppendParams p) {
   static_assert(NB >= 1 && NB <= kAppendBatch, "1..16 sequences per pass");
-  constexpr int kGroup = append_group(NB);          // steps per stage
-  constexpr int kAppendCols = kAppendStep * kGroup; // columns per stage
-  extern __shared__ __align__(16) float s_x[];  // [NB][kAppendCols]
-  __shared__ float s_part[kAppendWarps][NB][kAppendRows];
-  __shared__ __align__(16) uint16_t s_out[NB][kAppendRows];
+  constexpr int RL = append_rows_per_lane(NB);     // rows per lane: r and r + 8
+  constexpr int kRows = kAppendRows * RL;          // output rows of this CTA
+  constexpr int kGroup = append_group(NB);         // steps per stage
+  constexpr int kCols = kAppendStep * kGroup;      // columns per stage
+  extern __shared__ __align__(16) float s_x[];     // [NB][kCols]
+  __shared__ float s_part[kAppendWarps][NB][kRows];
+  __shared__ __align__(16) uint16_t s_out[NB][kRows];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int r = lane >> 2;                          // row of this lane among the CTA's 8
+  const int r = lane >> 2;                          // first row of this lane among the CTA's
   const int q = lane & 3;                           // its 16-byte column in the row's 64-byte run
   const int rows_kv = p.hkv * p.head_dim;
-  const int row0 = blockIdx.x * kAppendRows;        // first output row of this CTA
+  const int row0 = blockIdx.x * kRows;              // first output row of this CTA
   const bool is_v = row0 >= rows_kv;
   const int r_local = row0 - (is_v ? rows_kv : 0);  // row inside W_k or W_v
   const int h = r_local / p.head_dim;
-  const int d0 = r_local % p.head_dim;              // multiple of 8
-  const uint16_t* wrow = (is_v ? p.w_v : p.w_k) + static_cast<size_t>(r_local + r) * p.hidden;
+  const int d0 = r_local % p.head_dim;              // multiple of kRows
+  const uint16_t* wbase = (is_v ? p.w_v : p.w_k) + static_cast<size_t>(r_local + r) * p.hidden;
   const int col = (warp * 4 + q) * 8;               // this lane's 8 columns inside a step
-  auto load_w = [&](int c) {
-    return c < p.hidden ? *reinterpret_cast<const uint4*>(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+  auto load_w = [&](int j, int c) {                 // row r + 8j, columns c .. c+7
+    return c < p.hidden ? *reinterpret_cast<const uint4*>(wbase + static_cast<size_t>(8 * j) * p.hidden + c)
+                        : make_uint4(0u, 0u, 0u, 0u);
   };
 
   for (int b0 = 0; b0 < p.batch; b0 += NB) {
     const int nb = min(NB, p.batch - b0);
-    // destination of sequence b0 + threadIdx.x (threads < nb), looked up while
-    // the projection runs: its position, the table entry, the pool
+    // destination (dims d0 ..) of sequence b0 + threadIdx.x (threads < nb),
+    // looked up while the projection runs: its position, the table entry, the pool
     uint16_t* dst = nullptr;
     if (threadIdx.x < nb) {
       const int b = b0 + threadIdx.x;
@@ -141,19 +151,21 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 2) append_kernel(const Appe
         if (pool) dst = pool + ((blk * p.hkv + h) * p.block_size + (L % p.block_size)) * p.head_dim + d0;
       }
     }
-    // per sequence, even and odd columns accumulate in the two halves of a
-    // packed pair (one f32x2 FMA per two columns)
-    float2 acc[NB];
+    float acc[RL][NB];
 #pragma unroll
-    for (int i = 0; i < NB; ++i) acc[i] = make_float2(0.f, 0.f);
-    for (int g0 = 0; g0 < p.hidden; g0 += kAppendCols) {
+    for (int j = 0; j < RL; ++j)
+#pragma unroll
+      for (int i = 0; i < NB; ++i) acc[j][i] = 0.f;
+    for (int g0 = 0; g0 < p.hidden; g0 += kCols) {
       // this lane's weights of the stage, in flight while x is staged
-      uint4 raw[kGroup];
+      uint4 raw[RL][kGroup];
 #pragma unroll
-      for (int u = 0; u < kGroup; ++u) raw[u] = load_w(g0 + col + u * kAppendStep);
+      for (int u = 0; u < kGroup; ++u)
+#pragma unroll
+        for (int j = 0; j < RL; ++j) raw[j][u] = load_w(j, g0 + col + u * kAppendStep);
       // x of this stage (zeros for absent sequences and past the hidden size)
-      for (int e = threadIdx.x * 4; e < NB * kAppendCols; e += kAppendWarps * 32 * 4) {
-        const int i = e / kAppendCols, cc = e % kAppendCols;
+      for (int e = threadIdx.x * 4; e < NB * kCols; e += kAppendWarps * 32 * 4) {
+        const int i = e / kCols, cc = e % kCols;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (i < nb && g0 + cc < p.hidden)
           v = __ldg(reinterpret_cast<const float4*>(p.x + static_cast<size_t>(b0 + i) * p.hidden + g0 + cc));
@@ -162,36 +174,45 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 2) append_kernel(const Appe
       __syncthreads();
 #pragma unroll
       for (int u = 0; u < kGroup; ++u) {
-        float w[8];
-        widen8<BF16>(raw[u], w);   // zeros past the hidden size
-        const float2 w01 = make_float2(w[0], w[1]), w23 = make_float2(w[2], w[3]);
-        const float2 w45 = make_float2(w[4], w[5]), w67 = make_float2(w[6], w[7]);
+        float w[RL][8];
+#pragma unroll
+        for (int j = 0; j < RL; ++j) widen8<BF16>(raw[j][u], w[j]);   // zeros past the hidden size
         const int cs = col + u * kAppendStep;   // column inside the stage
 #pragma unroll
         for (int i = 0; i < NB; ++i) {
-          const float4 x0 = *reinterpret_cast<const float4*>(s_x + i * kAppendCols + cs);
-          const float4 x1 = *reinterpret_cast<const float4*>(s_x + i * kAppendCols + cs + 4);
-          float2 a = acc[i];
-          a = __ffma2_rn(w01, make_float2(x0.x, x0.y), a);
-          a = __ffma2_rn(w23, make_float2(x0.z, x0.w), a);
-          a = __ffma2_rn(w45, make_float2(x1.x, x1.y), a);
-          a = __ffma2_rn(w67, make_float2(x1.z, x1.w), a);
-          acc[i] = a;
+          const float4 x0 = *reinterpret_cast<const float4*>(s_x + i * kCols + cs);
+          const float4 x1 = *reinterpret_cast<const float4*>(s_x + i * kCols + cs + 4);
+#pragma unroll
+          for (int j = 0; j < RL; ++j) {
+            float a = acc[j][i];
+            a = fmaf(w[j][0], x0.x, a);
+            a = fmaf(w[j][1], x0.y, a);
+            a = fmaf(w[j][2], x0.z, a);
+            a = fmaf(w[j][3], x0.w, a);
+            a = fmaf(w[j][4], x1.x, a);
+            a = fmaf(w[j][5], x1.y, a);
+            a = fmaf(w[j][6], x1.z, a);
+            a = fmaf(w[j][7], x1.w, a);
+            acc[j][i] = a;
+          }
         }
       }
       __syncthreads();   // before the next stage overwrites s_x
     }
     // the 4 lanes of a row, then the warps
 #pragma unroll
-    for (int i = 0; i < NB; ++i) {
-      float a = acc[i].x + acc[i].y;
-      a += __shfl_xor_sync(0xffffffffu, a, 1);
-      a += __shfl_xor_sync(0xffffffffu, a, 2);
-      if (q == 0) s_part[warp][i][r] = a;
+    for (int j = 0; j < RL; ++j) {
+#pragma unroll
+      for (int i = 0; i < NB; ++i) {
+        float a = acc[j][i];
+        a += __shfl_xor_sync(0xffffffffu, a, 1);
+        a += __shfl_xor_sync(0xffffffffu, a, 2);
+        if (q == 0) s_part[warp][i][r + 8 * j] = a;
+      }
     }
     __syncthreads();
-    if (threadIdx.x < NB * kAppendRows) {
-      const int i = threadIdx.x / kAppendRows, rr = threadIdx.x % kAppendRows;
+    if (threadIdx.x < NB * kRows) {
+      const int i = threadIdx.x / kRows, rr = threadIdx.x % kRows;
       if (i < nb) {
         float a = 0.f;
 #pragma unroll
@@ -200,7 +221,11 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 2) append_kernel(const Appe
       }
     }
     __syncthreads();
-    if (dst) *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&s_out[threadIdx.x][0]);
+    if (dst) {
+#pragma unroll
+      for (int j = 0; j < RL; ++j)
+        *reinterpret_cast<uint4*>(dst + 8 * j) = *reinterpret_cast<const uint4*>(&s_out[threadIdx.x][8 * j]);
+    }
     __syncthreads();
   }
 }
