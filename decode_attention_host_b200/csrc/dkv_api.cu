@@ -195,13 +195,12 @@ size_t multi_smem(int D) { return dkv::multi_smem_bytes(D); }
 template <bool BF16, int NB>
 cudaError_t launch_append_nb(dim3 grid, cudaStream_t s, const dkv::AppendParams& ap) {
   const size_t smem = dkv::append_smem_bytes(NB);
-  if (smem > 48 * 1024) {
-    // once per process and instance (the attribute holds for every device)
-    static const cudaError_t set = cudaFuncSetAttribute(dkv::append_kernel<BF16, NB>,
-                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                        static_cast<int>(smem));
-    if (set != cudaSuccess) return set;
-  }
+  // once per process and instance (the attribute holds for every device): the
+  // kernel's static and dynamic shared memory together may pass 48 KB
+  static const cudaError_t set = cudaFuncSetAttribute(dkv::append_kernel<BF16, NB>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(smem));
+  if (set != cudaSuccess) return set;
   dkv::append_kernel<BF16, NB><<<grid, dkv::kAppendWarps * 32, smem, s>>>(ap);
   return cudaGetLastError();
 }

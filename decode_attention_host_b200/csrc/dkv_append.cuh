@@ -211,8 +211,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 2) append_kernel(const Appe
       }
     }
     __syncthreads();
-    if (threadIdx.x < NB * kRows) {
-      const int i = threadIdx.x / kRows, rr = threadIdx.x % kRows;
+    for (int t = threadIdx.x; t < NB * kRows; t += kAppendWarps * 32) {
+      const int i = t / kRows, rr = t % kRows;
       if (i < nb) {
         float a = 0.f;
 #pragma unroll
