@@ -9,12 +9,12 @@
 // holds position seq_lens[b], in the host or the device pool.
 //
 // The product is bound by the weight bytes (batch is small), so it runs on the
-// CUDA cores.  A CTA owns 8 consecutive output rows (8 dims of one head), so
-// each sequence's 8 results leave as one 16-byte store -- over PCIe when the
-// block is host-resident.  Its 8 warps split the hidden dimension: in each
-// warp, 4 lanes share a row and read a 64-byte run of it (16 bytes each), the
-// 8 rows side by side; every weight byte is read once for up to 16
-// sequences, whose hidden states the CTA stages in shared memory.  Lane
+// CUDA cores.  A CTA owns 8 consecutive output rows (16 with 16 sequences per
+// pass), dims of one head, so each sequence's results leave as 16-byte stores
+// -- over PCIe when the block is host-resident.  Its 8 warps split the hidden
+// dimension: in each warp, 4 lanes share a row and read a 64-byte run of it
+// (16 bytes each), 8 rows side by side; every weight byte is read once for up
+// to 16 sequences, whose hidden states the CTA stages in shared memory.  Lane
 // partials are combined by shuffles, the warps' through shared memory.
 #pragma once
 
@@ -25,7 +25,7 @@
 
 namespace dkv {
 
-constexpr int kAppendRows = 8;                 // rows one lane of each of 8 row slots covers per CTA
+constexpr int kAppendRows = 8;                 // row slots of a CTA (lane / 4); a lane covers 1 or 2 rows
 constexpr int kAppendWarps = 8;                // warps per CTA, each over part of the hidden dimension
 constexpr int kAppendBatch = 16;               // sequences per pass over the weights
 
