@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 import subprocess
+from pathlib import Path
 
 import numpy as np
 import pytest
@@ -99,3 +100,34 @@ def test_null_arguments_are_rejected():
     assert dkv.lib.dkv_host_pool_alloc(0, None) == dkv.DKV_ERR_INVALID_ARG
     assert dkv.lib.dkv_destroy(None) == dkv.DKV_OK
     assert dkv.lib.dkv_host_pool_free(None) == dkv.DKV_OK
+
+
+def test_a_c_program_links_and_calls_the_host_entry_points(tmp_path):
+    """A plain C11 program built against include/dkv.h and linked to libdkv.so: the host-only entry points
+    answer through their declared prototypes (no GPU needed)."""
+    src = tmp_path / "consumer.c"
+    src.write_text(r"""
+#include <math.h>
+#include <stdio.h>
+#include "dkv.h"
+int main(void) {
+  dkv_offload_plan plan;
+  /* 4 GiB, 51 GB/s host, 4500 GB/s beside the host stream, unlimited budget, 5600 GB/s alone */
+  if (dkv_plan_offload(4294967296.0, 51.0, 4500.0, -1.0, 5600.0, &plan) != DKV_OK) return 1;
+  if (plan.host_fraction != 0.0) return 2;
+  if (fabs(plan.step_seconds - 4294967296.0 / 5600e9) > 1e-15) return 3;
+  if (dkv_plan_offload(4294967296.0, 51.0, 4500.0, 0.5 * 4294967296.0, 5600.0, &plan) != DKV_OK) return 4;
+  if (fabs(plan.host_fraction - 0.5) > 1e-12) return 5;
+  if (dkv_plan_offload(0.0, 51.0, 4500.0, -1.0, -1.0, &plan) != DKV_ERR_INVALID_ARG) return 6;
+  if (dkv_last_error_string()[0] == '\0') return 7;
+  if (dkv_create(NULL, NULL) != DKV_ERR_INVALID_ARG) return 8;
+  printf("ok\n");
+  return 0;
+}
+""")
+    exe = tmp_path / "consumer"
+    lib = Path(dkv.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", f"-I{ROOT}/include", "-o", str(exe), str(src), str(lib),
+                    f"-Wl,-rpath,{lib.parent}", "-lm"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
