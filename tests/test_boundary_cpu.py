@@ -6,7 +6,6 @@ import re
 import subprocess
 from pathlib import Path
 
-import numpy as np
 import pytest
 
 import decode_attention_host_b200 as dkv

@@ -1,8 +1,6 @@
 """Per-kernel attribution on the GPU: the events the library records around each kernel, the per-call timeline
 (which shows the host-stream and HBM kernels overlapping) and the launch counts."""
-import numpy as np
 import pytest
-import torch
 
 import decode_attention_host_b200 as dkv
 import kvgen

@@ -4,7 +4,6 @@ Each mutant is the oracle's C source with one textual change, compiled into a
 temporary directory on the CPU.  A mutant that passes every pin would mean
 the pins cannot tell that mistake from the right answer.
 """
-import ctypes
 
 import pytest
 
